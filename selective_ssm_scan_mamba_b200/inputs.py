@@ -1,0 +1,155 @@
+"""Seeded synthetic inputs for the block-confined bidirectional selective scan.
+
+This module is the one piece shared by the CUDA path's tests/bench and the CPU
+oracle: it only draws random numbers and rounds them to the storage dtype. It
+holds none of the scan's arithmetic.
+
+Workloads follow the five configurations of the block-diffusion Mamba-H mixer
+workloads (value distributions of the mixer inputs):
+
+* ``x ~ N(0, 1)``                    ``[batch, L, D]``   (io dtype)
+* ``dt_raw ~ N(-2, 0.5)``            ``[batch, L, D]``   (io dtype; the kernel
+  applies ``softplus`` itself, so the stored operand is the raw value)
+* ``A = -exp(U(log 1, log 16))``     ``[D, N]``          fp32
+* ``B, C ~ N(0, 1) / sqrt(N)``       ``[batch, L, N]``   (io dtype)
+* ``Dskip ~ N(0, 1)``                ``[D]``             fp32
+* ``z ~ N(0, 1)``                    ``[batch, L, D]``   (optional gate)
+
+Random streams are keyed, not sequential: every (array, stream, batch row,
+4096-token chunk) draws from its own ``PCG64(SeedSequence([seed, ...key]))``.
+Any token range of any batch row is therefore reproducible on its own, which
+lets a test regenerate a slice of a 262,144-token context without holding the
+whole context in host memory, and lets the oracle see exactly the values the
+GPU saw. bf16 values are produced by round-to-nearest-even from the fp32 draw
+and returned as their raw ``uint16`` bit patterns.
+"""
+from __future__ import annotations
+
+import dataclasses
+import numpy as np
+
+CHUNK = 4096  # tokens per independently seeded chunk
+
+_ARRAY_IDS = {"x": 1, "dt": 2, "B": 3, "C": 4, "z": 5, "A": 6, "Dskip": 7}
+# streams name independent sequences inside one workload
+_STREAM_IDS = {"seq": 0, "context": 1, "noisy": 2, "clean": 3, "layer": 4}
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Round fp32 to bf16 (round to nearest, ties to even); returns uint16 bits."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    u = a.view(np.uint32).astype(np.uint64)
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return rounded.astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to fp32."""
+    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def _rng(seed: int, *key: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([int(seed), *map(int, key)])))
+
+
+def _stream_key(stream) -> tuple:
+    if isinstance(stream, str):
+        stream = (stream,)
+    name, *rest = stream
+    return (_STREAM_IDS[name], *[int(r) for r in rest])
+
+
+def _draw_rows(seed, array, stream, b, t0, t1, width, mean, std):
+    """fp32 draws for tokens [t0, t1) of batch row b, assembled from fixed chunks."""
+    out = np.empty((t1 - t0, width), dtype=np.float32)
+    c0, c1 = t0 // CHUNK, (t1 - 1) // CHUNK if t1 > t0 else t0 // CHUNK - 1
+    for c in range(c0, c1 + 1):
+        g = _rng(seed, _ARRAY_IDS[array], *_stream_key(stream), b, c)
+        blk = g.standard_normal((CHUNK, width), dtype=np.float32)
+        if std != 1.0:
+            blk *= np.float32(std)
+        if mean != 0.0:
+            blk += np.float32(mean)
+        lo, hi = max(t0, c * CHUNK), min(t1, (c + 1) * CHUNK)
+        out[lo - t0:hi - t0] = blk[lo - c * CHUNK:hi - c * CHUNK]
+    return out
+
+
+def _cast(a32: np.ndarray, io: str) -> np.ndarray:
+    if io == "bf16":
+        return f32_to_bf16_bits(a32)
+    if io == "f32":
+        return np.ascontiguousarray(a32, dtype=np.float32)
+    raise ValueError(f"io dtype {io!r}")
+
+
+def make_sequence(seed: int, batch: int, L: int, D: int, N: int, io: str,
+                  stream="seq", t0: int = 0, gated: bool = False,
+                  channels=None) -> dict:
+    """Per-token inputs x, dt, B, C (and z) for tokens [t0, t0+L) of `stream`.
+
+    ``channels`` optionally restricts x/dt/z to a subset of channel indices
+    (B and C are shared by all channels and always returned whole).
+    """
+    t1 = t0 + L
+    out = {k: [] for k in (("x", "dt", "B", "C", "z") if gated else ("x", "dt", "B", "C"))}
+    for b in range(batch):
+        for name, width, mean, std in (("x", D, 0.0, 1.0), ("dt", D, -2.0, 0.5),
+                                       ("B", N, 0.0, 1.0 / np.sqrt(N)),
+                                       ("C", N, 0.0, 1.0 / np.sqrt(N)),
+                                       ("z", D, 0.0, 1.0)):
+            if name not in out:
+                continue
+            rows = _draw_rows(seed, name, stream, b, t0, t1, width, mean, std)
+            if channels is not None and name in ("x", "dt", "z"):
+                rows = rows[:, channels]
+            out[name].append(_cast(rows, io))
+    return {k: np.ascontiguousarray(np.stack(v)) for k, v in out.items()}
+
+
+def make_params(seed: int, D: int, N: int, layer: int = 0) -> dict:
+    """Per-channel parameters: A [D, N] fp32 (negative) and Dskip [D] fp32."""
+    g = _rng(seed, _ARRAY_IDS["A"], _STREAM_IDS["layer"], layer)
+    u = g.uniform(np.log(1.0), np.log(16.0), size=(D, N))
+    A = (-np.exp(u)).astype(np.float32)
+    g = _rng(seed, _ARRAY_IDS["Dskip"], _STREAM_IDS["layer"], layer)
+    Dskip = g.standard_normal(D).astype(np.float32)
+    return {"A": np.ascontiguousarray(A), "Dskip": np.ascontiguousarray(Dskip)}
+
+
+def make_state(seed: int, batch: int, D: int, N: int, scale: float = 1.0) -> np.ndarray:
+    """A generic fp32 initial state [batch, D, N] ~ N(0, scale^2) for tests."""
+    g = _rng(seed, 99, batch, D, N)
+    return (g.standard_normal((batch, D, N)) * scale).astype(np.float32)
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One of the five mixer workloads (sizes, block length, dtype, seed)."""
+    name: str
+    batch: int
+    L: int            # tokens scanned by the main call (train / prefill)
+    D: int
+    N: int
+    K: int            # block length
+    io: str
+    seed: int
+    steps: int = 0    # denoising steps per block (inference workloads)
+    blocks: int = 0   # committed blocks (inference workloads)
+    layers: int = 1
+    note: str = ""
+
+
+WORKLOADS = {
+    "pr1": Workload("pr1", batch=1, L=256, D=64, N=16, K=16, io="f32", seed=0,
+                    note="one mixer, 16 block-boundary states, fp32"),
+    "train": Workload("train", batch=8, L=4096, D=1536, N=16, K=16, io="bf16", seed=1,
+                      note="full-block training objective, all blocks in one launch"),
+    "step65k": Workload("step65k", batch=1, L=65536, D=1536, N=16, K=32, io="bf16", seed=2,
+                        steps=32, blocks=1, note="block step at a 65,536-token context"),
+    "step262k": Workload("step262k", batch=4, L=262144, D=2048, N=16, K=32, io="bf16", seed=3,
+                         steps=64, blocks=8, note="block steps at a 262,144-token context"),
+    "stack350m": Workload("stack350m", batch=16, L=8192, D=2048, N=64, K=16, io="bf16", seed=4,
+                          layers=24, note="24 mixer layers, block sizes {4,16,64,256}"),
+}
+STACK_BLOCK_SIZES = (4, 16, 64, 256)

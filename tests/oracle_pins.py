@@ -1,0 +1,240 @@
+"""Pins for the CPU oracle: checks against facts that do not come from the
+oracle itself (a hand-derived example, closed forms, an independent matrix
+evaluation, and the invariants the method states).
+
+Each check takes the oracle build to test (``mutant`` = 0 is the real one;
+1..7 are builds with one planted mistake) and returns ``(ok, detail)``, so the
+same checks both pin the real oracle and prove that each planted mistake is
+caught.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+import oracle
+from selective_ssm_scan_mamba_b200 import inputs as I
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+LN2, LN3 = math.log(2.0), math.log(3.0)
+
+
+def _val(v):
+    if isinstance(v, str):
+        return float(eval(v, {"ln2": LN2, "ln3": LN3}))  # fixture expressions only
+    p, q = v
+    return p * LN2 + q
+
+
+def _close(a, b, rtol=1e-12, atol=1e-12):
+    a, b = np.asarray(a, dtype=np.float64), np.asarray(b, dtype=np.float64)
+    return a.shape == b.shape and bool(np.all(np.abs(a - b) <= atol + rtol * np.abs(b)))
+
+
+def _small(seed, Bt, L, D, N, io="f32", gated=False):
+    s = I.make_sequence(seed, Bt, L, D, N, io, gated=gated)
+    s.update(I.make_params(seed, D, N))
+    return s
+
+
+# ---------------------------------------------------------------- hand example
+def check_hand_example(mutant=0):
+    g = json.load(open(os.path.join(GOLDEN, "hand_example.json")))
+    inp = g["inputs"]
+    A = np.array(inp["A"], dtype=np.float64)
+    B = np.array(inp["B"], dtype=np.float64).reshape(1, 2, 1)
+    C = np.array(inp["C"], dtype=np.float64).reshape(1, 2, 1)
+    x = np.array(inp["x"], dtype=np.float64).reshape(1, 2, 1)
+    Dskip = np.array(inp["Dskip"], dtype=np.float64)
+    delta = np.array([_val(v) for v in inp["delta"]]).reshape(1, 2, 1)
+    raw = np.array([_val(v) for v in inp["dt_raw_softplus"]]).reshape(1, 2, 1)
+    for case in g["cases"]:
+        K = case["K"]
+        h0 = None if case["h0"] is None else np.full((1, 1, 1), case["h0"])
+        z = None if case["z"] is None else np.array([_val(v) for v in case["z"]]).reshape(1, 2, 1)
+        for dt, sp in ((delta, False), (raw, True)):
+            f = oracle.forward(x, dt, A, B, C, Dskip, K, h0=h0, dt_softplus=sp, mutant=mutant)
+            r = oracle.reverse_blocks(x, dt, A, B, C, Dskip, K, dt_softplus=sp, mutant=mutant)
+            y = oracle.train_blocks(x, dt, A, B, C, Dskip, K, z=z, h0=h0, dt_softplus=sp, mutant=mutant)
+            want = lambda key: np.array([_val(v) for v in case[key]])  # noqa: E731
+            if "y_fwd" in case and not _close(f["y_fwd"].ravel(), want("y_fwd")):
+                return False, f"y_fwd K={K} softplus={sp}: {f['y_fwd'].ravel()} vs {want('y_fwd')}"
+            if "y_rev" in case and not _close(r.ravel(), want("y_rev")):
+                return False, f"y_rev K={K} softplus={sp}: {r.ravel()} vs {want('y_rev')}"
+            if not _close(y["y"].ravel(), want("y")):
+                return False, f"y K={K} softplus={sp}: {y['y'].ravel()} vs {want('y')}"
+            if "boundary" in case and not _close(f["boundary"].ravel(), want("boundary")):
+                return False, f"boundary K={K}: {f['boundary'].ravel()} vs {want('boundary')}"
+            if "h_out" in case and not _close(f["h_out"].ravel(), [_val(case["h_out"])]):
+                return False, f"h_out K={K}"
+    return True, ""
+
+
+# ----------------------------------------------------------------- closed forms
+def check_softplus_closed_forms(mutant=0):
+    sp = lambda v: oracle.softplus(v, mutant)  # noqa: E731
+    cases = [(0.0, LN2), (LN3, 2 * LN2), (math.log(math.e - 1.0), 1.0),
+             (-40.0, math.exp(-40.0)), (40.0, 40.0 + math.exp(-40.0))]
+    for v, want in cases:
+        got = sp(v)
+        if not abs(got - want) <= 1e-14 * abs(want):
+            return False, f"softplus({v}) = {got}, want {want}"
+    return True, ""
+
+
+def check_block1_closed_form(mutant=0):
+    """K = 1: the reverse term is delta * x * (C . B) + Dskip * x at every token."""
+    s = _small(11, 2, 12, 5, 4)
+    y_rev = oracle.reverse_blocks(s["x"], s["dt"], s["A"], s["B"], s["C"], s["Dskip"], 1, mutant=mutant)
+    x = s["x"].astype(np.float64)
+    raw = s["dt"].astype(np.float64)
+    delta = np.maximum(raw, 0) + np.log1p(np.exp(-np.abs(raw)))
+    cb = np.einsum("btn,btn->bt", s["C"].astype(np.float64), s["B"].astype(np.float64))
+    want = delta * x * cb[:, :, None] + s["Dskip"].astype(np.float64)[None, None, :] * x
+    return _close(y_rev, want, rtol=1e-12, atol=1e-13), "K=1 reverse closed form"
+
+
+def check_blockL_flip(mutant=0):
+    """K = L: the reverse term equals the forward scan of the time-reversed inputs (zero state)."""
+    s = _small(12, 2, 24, 3, 5)
+    y_rev = oracle.reverse_blocks(s["x"], s["dt"], s["A"], s["B"], s["C"], s["Dskip"], 24, mutant=mutant)
+    fl = {k: np.ascontiguousarray(s[k][:, ::-1]) for k in ("x", "dt", "B", "C")}
+    f = oracle.forward(fl["x"], fl["dt"], s["A"], fl["B"], fl["C"], s["Dskip"], 24, mutant=mutant)
+    ok = _close(y_rev, f["y_fwd"][:, ::-1], rtol=1e-12, atol=1e-13)
+    # per-block flip for K < L
+    K = 6
+    y_rev = oracle.reverse_blocks(s["x"], s["dt"], s["A"], s["B"], s["C"], s["Dskip"], K, mutant=mutant)
+    for j in range(24 // K):
+        sl = slice(j * K, (j + 1) * K)
+        fl = {k: np.ascontiguousarray(s[k][:, sl][:, ::-1]) for k in ("x", "dt", "B", "C")}
+        f = oracle.forward(fl["x"], fl["dt"], s["A"], fl["B"], fl["C"], s["Dskip"], K, mutant=mutant)
+        ok = ok and _close(y_rev[:, sl], f["y_fwd"][:, ::-1], rtol=1e-12, atol=1e-13)
+    return ok, "reverse == flipped forward"
+
+
+def check_bruteforce(mutant=0):
+    """Recurrence vs explicit matrix form, every L in 1..8 and every K dividing L."""
+    for L in range(1, 9):
+        for K in [k for k in range(1, L + 1) if L % k == 0]:
+            for gated, with_h0, sp in ((False, False, True), (True, True, True), (False, True, False)):
+                s = _small(100 + L * 10 + K, 2, L, 3, 3, gated=gated)
+                dt = s["dt"] if sp else np.abs(s["dt"]) * np.float32(0.3)
+                h0 = I.make_state(L * 7 + K, 2, 3, 3) if with_h0 else None
+                r = oracle.train_blocks(s["x"], dt, s["A"], s["B"], s["C"], s["Dskip"], K,
+                                        z=s.get("z"), h0=h0, dt_softplus=sp, mutant=mutant)
+                bf = oracle.bruteforce(s["x"], dt, s["A"], s["B"], s["C"], s["Dskip"], K,
+                                       z=s.get("z"), h0=h0, dt_softplus=sp)
+                if not _close(r["y"], bf["y"], rtol=1e-11, atol=1e-12):
+                    return False, f"y L={L} K={K} gated={gated} h0={with_h0} sp={sp}"
+                if not _close(r["boundary"], bf["boundary"], rtol=1e-11, atol=1e-12):
+                    return False, f"boundary L={L} K={K}"
+    return True, ""
+
+
+def check_steady_state(mutant=0):
+    """Constant inputs: the forward state converges to the geometric-series limit
+    h = delta x B / (1 - exp(delta A))."""
+    L, D, N = 400, 2, 3
+    x = np.full((1, L, D), 0.75, np.float32)
+    dt = np.full((1, L, D), 0.25, np.float32)
+    A = -np.array([[1.0, 2.0, 5.0], [0.5, 3.0, 8.0]], np.float32)
+    B = np.tile(np.array([0.25, -0.125, 0.875], np.float32), (1, L, 1))
+    C = np.tile(np.array([1.0, 0.5, -0.25], np.float32), (1, L, 1))
+    Dskip = np.array([0.5, -0.25], np.float32)
+    f = oracle.forward(x, dt, A, B, C, Dskip, L, dt_softplus=False, mutant=mutant)
+    d, a = 0.25, np.exp(0.25 * A.astype(np.float64))
+    h_inf = d * 0.75 * B[0, 0].astype(np.float64)[None, :] / (1.0 - a)
+    ok = _close(f["h_out"][0], h_inf, rtol=1e-12)
+    y_inf = h_inf @ C[0, 0].astype(np.float64) + Dskip.astype(np.float64) * 0.75
+    ok = ok and _close(f["y_fwd"][0, -1], y_inf, rtol=1e-12)
+    # reverse within a long block also converges (at its start) to the same limit
+    r = oracle.reverse_blocks(x, dt, A, B, C, Dskip, L, dt_softplus=False, mutant=mutant)
+    ok = ok and _close(r[0, 0], y_inf, rtol=1e-12)
+    return ok, "steady state"
+
+
+def check_linearity(mutant=0):
+    s = _small(13, 1, 16, 4, 4, gated=False)
+    x1, x2 = s["x"], I.make_sequence(14, 1, 16, 4, 4, "f32")["x"]
+    al, be = 0.75, -1.5
+    x3 = (al * x1.astype(np.float64) + be * x2.astype(np.float64))
+    run = lambda x: oracle.train_blocks(x, s["dt"], s["A"], s["B"], s["C"], s["Dskip"], 4, mutant=mutant)["y"]  # noqa: E731
+    return _close(run(x3), al * run(x1) + be * run(x2), rtol=1e-12, atol=1e-12), "linearity"
+
+
+def check_zero_limits(mutant=0):
+    s = _small(15, 2, 8, 3, 4)
+    z = np.zeros_like(s["x"])
+    r = oracle.train_blocks(z, s["dt"], s["A"], s["B"], s["C"], s["Dskip"], 4, mutant=mutant)
+    if np.any(r["y"] != 0):
+        return False, "x=0, h0=0 must give y=0"
+    h0 = I.make_state(3, 2, 3, 4)
+    f = oracle.forward(z, s["dt"], s["A"], s["B"], s["C"], s["Dskip"], 4, h0=h0, mutant=mutant)
+    rv = oracle.reverse_blocks(z, s["dt"], s["A"], s["B"], s["C"], s["Dskip"], 4, mutant=mutant)
+    if np.any(rv != 0):
+        return False, "x=0: reverse term must vanish"
+    raw = s["dt"].astype(np.float64)
+    delta = np.maximum(raw, 0) + np.log1p(np.exp(-np.abs(raw)))
+    S = np.cumsum(delta, axis=1)  # [Bt, L, D]
+    decay = np.exp(S[:, :, :, None] * s["A"].astype(np.float64)[None, None])  # prod_{r<=t} a_r
+    want = np.einsum("btn,btdn,bdn->btd", s["C"].astype(np.float64), decay, h0.astype(np.float64))
+    return _close(f["y_fwd"], want, rtol=1e-12, atol=1e-14), "x=0: pure decay of h0"
+
+
+# ------------------------------------------------------------------ invariants
+def check_commit_chain(mutant=0):
+    """Cache exactness: committing blocks one after another reproduces, bit for
+    bit, the boundary states of a one-shot scan of the whole clean sequence."""
+    Bt, L, D, N, K = 2, 40, 3, 4, 8
+    s = _small(16, Bt, L, D, N)
+    one = oracle.prefill(s["x"], s["dt"], s["A"], s["B"], s["C"], s["Dskip"], K, mutant=mutant)
+    h = np.zeros((Bt, D, N))
+    for j in range(L // K):
+        sl = slice(j * K, (j + 1) * K)
+        blk = {k: np.ascontiguousarray(s[k][:, sl]) for k in ("x", "dt", "B", "C")}
+        h, _ = oracle.commit_block(blk["x"], blk["dt"], s["A"], blk["B"], blk["C"], s["Dskip"], h, mutant=mutant)
+        if not np.array_equal(h, one["boundary"][:, j]):
+            return False, f"commit {j} differs from one-shot boundary state"
+    return np.array_equal(h, one["h_out"]), "commit chain"
+
+
+def check_prefix_only(mutant=0):
+    """Boundary state k depends only on tokens before it."""
+    Bt, L, D, N, K = 1, 32, 3, 4, 8
+    s = _small(17, Bt, L, D, N)
+    base = oracle.forward(s["x"], s["dt"], s["A"], s["B"], s["C"], s["Dskip"], K, mutant=mutant)["boundary"]
+    for k in range(1, L // K):
+        p = {kk: s[kk].copy() for kk in ("x", "dt", "B", "C")}
+        for kk in p:
+            p[kk][:, k * K:] = p[kk][:, k * K:][:, ::-1] * np.float32(1.5)
+        pb = oracle.forward(p["x"], p["dt"], s["A"], p["B"], p["C"], s["Dskip"], K, mutant=mutant)["boundary"]
+        if not np.array_equal(pb[:, :k], base[:, :k]):
+            return False, f"boundary states before {k} changed"
+    return True, ""
+
+
+def check_block_locality(mutant=0):
+    """The reverse term of block j depends only on the tokens of block j."""
+    Bt, L, D, N, K = 1, 32, 3, 4, 8
+    s = _small(18, Bt, L, D, N)
+    base = oracle.reverse_blocks(s["x"], s["dt"], s["A"], s["B"], s["C"], s["Dskip"], K, mutant=mutant)
+    for j in range(L // K):
+        p = {kk: s[kk].copy() for kk in ("x", "dt", "B", "C")}
+        mask = np.ones(L, bool)
+        mask[j * K:(j + 1) * K] = False
+        for kk in p:
+            p[kk][:, mask] = -p[kk][:, mask] * np.float32(2.0) + np.float32(0.25)
+        pr = oracle.reverse_blocks(p["x"], p["dt"], s["A"], p["B"], p["C"], s["Dskip"], K, mutant=mutant)
+        if not np.array_equal(pr[:, j * K:(j + 1) * K], base[:, j * K:(j + 1) * K]):
+            return False, f"block {j} reverse term depends on other blocks"
+    return True, ""
+
+
+ALL_CHECKS = [
+    check_hand_example, check_softplus_closed_forms, check_block1_closed_form, check_blockL_flip,
+    check_bruteforce, check_steady_state, check_linearity, check_zero_limits, check_commit_chain,
+    check_prefix_only, check_block_locality,
+]
