@@ -1,0 +1,150 @@
+/*
+ * bdscan.h: C ABI of the block-confined bidirectional selective scan, the
+ * Mamba mixer of BDLM Mamba-H, running on NVIDIA B200 (sm_100a).
+ *
+ * Source of the method: "Training Hybrid Block Diffusion Language Models with
+ * Partial Bidirectionality" (arXiv 2607.02805).
+ *   - Abstract: the reverse Mamba scan is restricted to the active denoising
+ *     block, which enables exact caching across blocks.
+ *   - gist.science technical summary, "Methodik" (cache-aligned objective):
+ *     Mamba layers cache only forward boundary states; the reverse scan is
+ *     confined to the active block, so the prefix cache depends on the clean
+ *     prefix alone.
+ *   - same summary, "Wesentliche Beitraege": the objects cached by the
+ *     all-block training objective equal the inference-time block caches.
+ *
+ * The pages never write the recurrence. This library computes the standard
+ * Mamba selective scan in both directions, with shared parameters:
+ *   delta_t = softplus(dt_t)  (dims.dt_softplus = 1)  or  dt_t  (= 0)
+ *   a_t[n]  = exp(delta_t * A[d,n]),   b_t[n] = delta_t * x_t * B_t[n]
+ *   forward   h_t = a_t * h_{t-1} + b_t            (h_{-1} = h0 or the cache)
+ *             y_fwd_t = sum_n C_t[n] h_t[n] + Dskip[d] x_t
+ *   reverse   g_t = a_t * g_{t+1} + b_t  inside each block [jK, (j+1)K),
+ *             g = 0 after the block's last token
+ *             y_rev_t = sum_n C_t[n] g_t[n] + Dskip[d] x_t
+ *   output    y_t = (y_fwd_t + y_rev_t) * (z ? silu(z_t) : 1)
+ * (y therefore carries Dskip * x twice.) The forward state at the end of a
+ * block is the cache for the next block.
+ *
+ * Data layout, all row-major and contiguous, on the device:
+ *   x, dt, z, y   [batch, L, D]        io dtype (fp32 or bf16)
+ *   B, C          [batch, L, N]        io dtype
+ *   A             [D, N]               fp32 (negative for a decaying state)
+ *   Dskip         [D]                  fp32
+ *   h0, h_out, h_cache  [batch, D, N]  fp32
+ *   boundary      [batch, L/K, D, N]   fp32, the state after each block's
+ *                                      last token (the last one equals h_out)
+ *
+ * Conventions shared by every entry point:
+ *   - All pointers are device pointers owned by the caller; the library
+ *     allocates nothing, keeps no global device state and never synchronises.
+ *     Work is queued on `stream` (NULL = the legacy default stream) and the
+ *     call returns without waiting for it.
+ *   - Every pointer must be 16-byte aligned. D must be a multiple of 8 for
+ *     bf16 and of 4 for fp32; N must be 16 or 64; L must be a multiple of K.
+ *     A pointer may be NULL only when its tensor has no elements (for
+ *     example x when L == 0).
+ *   - Arguments are checked before anything is queued. A call that returns an
+ *     error has queued nothing, except BDSCAN_ERR_CUDA, which reports a failed
+ *     launch (the launch error is then also left in the CUDA runtime).
+ *   - Results are deterministic: the same inputs give bit-identical outputs.
+ *   - Input and output buffers must not overlap, except h_cache in
+ *     bdscan_commit_block, which is read and written in place.
+ */
+#ifndef BDSCAN_H
+#define BDSCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                        /* the CUDA runtime's cudaStream_t */
+typedef struct CUstream_st *bdscan_stream_t;
+
+typedef enum {
+    BDSCAN_OK = 0,
+    BDSCAN_ERR_INVALID_ARG = 1,  /* NULL required pointer, negative size, L % K != 0, ... */
+    BDSCAN_ERR_UNSUPPORTED = 2,  /* N not 16/64, D not a multiple of the vector width,
+                                    K > 768 for a pass with a reverse scan */
+    BDSCAN_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned */
+    BDSCAN_ERR_CUDA = 5          /* a kernel launch failed; see bdscan_last_cuda_error() */
+} bdscan_status;
+
+typedef enum { BDSCAN_F32 = 0, BDSCAN_BF16 = 1 } bdscan_dtype;
+
+typedef struct {
+    int64_t batch;        /* independent sequences in the call */
+    int64_t seqlen;       /* L, tokens in the call (block_step / commit: L == K) */
+    int64_t d_inner;      /* D, channels */
+    int64_t d_state;      /* N, state size per channel: 16 or 64 */
+    int64_t block;        /* K, denoising block length, K >= 1, L % K == 0 */
+    int32_t io_dtype;     /* bdscan_dtype of x, dt, B, C, z and y */
+    int32_t dt_softplus;  /* 1: delta = softplus(dt); 0: delta = dt */
+} bdscan_dims;
+
+typedef struct {
+    const void *x;        /* [batch, L, D] */
+    const void *dt;       /* [batch, L, D] raw step (softplus applied in-kernel if asked) */
+    const void *B;        /* [batch, L, N] */
+    const void *C;        /* [batch, L, N] */
+    const void *z;        /* [batch, L, D] gate input, or NULL for no gate */
+    const float *A;       /* [D, N] */
+    const float *Dskip;   /* [D] */
+} bdscan_inputs;
+
+/* Full-block (all-block) training pass: every block of every sequence in one
+ * launch. Forward scan over all L tokens from h0 (NULL = zero state) plus the
+ * block-confined reverse scan of each block; y = (y_fwd + y_rev) * gate.
+ * Optional outputs: boundary states after each block (NULL = not written) and
+ * the final state h_out (NULL = not written). Blocks longer than 32 tokens
+ * take a two-sweep path that stages the block's reverse readout in shared
+ * memory, which limits K to 768; longer blocks return BDSCAN_ERR_UNSUPPORTED.
+ * Source: full-block objective, gist.science technical summary, "Methodik";
+ * cache agreement, "Wesentliche Beitraege". */
+int bdscan_train_blocks(const bdscan_dims *dims, const bdscan_inputs *in,
+                        const float *h0, void *y, float *boundary, float *h_out,
+                        bdscan_stream_t stream);
+
+/* Forward-only scan of a clean context (the prefix operator): h_out receives
+ * the final state (required); y = y_fwd * gate if y is not NULL; boundary
+ * states after every K tokens if boundary is not NULL (K only matters there).
+ * Source: forward-only Mamba boundary states, gist.science technical summary,
+ * "Methodik". */
+int bdscan_prefill(const bdscan_dims *dims, const bdscan_inputs *in,
+                   const float *h0, void *y, float *h_out, float *boundary,
+                   bdscan_stream_t stream);
+
+/* One denoising step of the active block (dims.seqlen == dims.block): forward
+ * scan resumed from h_cache plus the in-block reverse scan from zero;
+ * y = (y_fwd + y_rev) * gate. h_cache is only read.
+ * Source: abstract (reverse scan restricted to the active block; exact cache
+ * reuse across blocks). */
+int bdscan_block_step(const bdscan_dims *dims, const bdscan_inputs *in,
+                      const float *h_cache, void *y, bdscan_stream_t stream);
+
+/* Commit a finished block (dims.seqlen == dims.block) with its clean inputs:
+ * h_cache is advanced in place to the forward state after the block's last
+ * token. If y is not NULL it receives what bdscan_block_step would return on
+ * these inputs. Source: exact caching across blocks, abstract; cache built by
+ * scanning the clean prefix, gist.science technical summary, "Methodik". */
+int bdscan_commit_block(const bdscan_dims *dims, const bdscan_inputs *in,
+                        float *h_cache, void *y, bdscan_stream_t stream);
+
+/* Human-readable name of a bdscan_status value (static storage). */
+const char *bdscan_status_string(int status);
+
+/* Text of the CUDA error behind the calling thread's last BDSCAN_ERR_CUDA
+ * (static storage; "no error" if none). */
+const char *bdscan_last_cuda_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int bdscan_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BDSCAN_H */

@@ -1,0 +1,192 @@
+"""Python binding of ``libbdscan.so`` (C ABI in ``include/bdscan.h``).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, output tensors are allocated with PyTorch when the caller does not
+pass them, and the call is queued on PyTorch's current CUDA stream. Every step
+of the scan runs in the library's CUDA kernels; there is no other code path.
+If the library has not been built this module fails to import.
+"""
+from __future__ import annotations
+
+import ctypes as ct
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libbdscan.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m selective_ssm_scan_mamba_b200.build`")
+_lib = ct.CDLL(_LIB_PATH)
+
+F32, BF16 = 0, 1
+_STATUS = {0: "BDSCAN_OK", 1: "BDSCAN_ERR_INVALID_ARG", 2: "BDSCAN_ERR_UNSUPPORTED",
+           3: "BDSCAN_ERR_ALIGNMENT", 5: "BDSCAN_ERR_CUDA"}
+
+
+class Dims(ct.Structure):
+    _fields_ = [("batch", ct.c_int64), ("seqlen", ct.c_int64), ("d_inner", ct.c_int64),
+                ("d_state", ct.c_int64), ("block", ct.c_int64), ("io_dtype", ct.c_int32),
+                ("dt_softplus", ct.c_int32)]
+
+
+class Inputs(ct.Structure):
+    _fields_ = [("x", ct.c_void_p), ("dt", ct.c_void_p), ("B", ct.c_void_p), ("C", ct.c_void_p),
+                ("z", ct.c_void_p), ("A", ct.c_void_p), ("Dskip", ct.c_void_p)]
+
+
+_vp = ct.c_void_p
+_P = ct.POINTER
+_lib.bdscan_train_blocks.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp, _vp, _vp]
+_lib.bdscan_prefill.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp, _vp, _vp]
+_lib.bdscan_block_step.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp]
+_lib.bdscan_commit_block.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp]
+for _f in ("bdscan_train_blocks", "bdscan_prefill", "bdscan_block_step", "bdscan_commit_block",
+           "bdscan_version"):
+    getattr(_lib, _f).restype = ct.c_int
+_lib.bdscan_status_string.argtypes = [ct.c_int]
+_lib.bdscan_status_string.restype = ct.c_char_p
+_lib.bdscan_last_cuda_error.restype = ct.c_char_p
+
+LIBRARY_PATH = _LIB_PATH
+version = _lib.bdscan_version
+
+
+class BdscanError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = f"{where}: {_lib.bdscan_status_string(status).decode()}"
+        if status == 5:
+            msg += f" ({_lib.bdscan_last_cuda_error().decode()})"
+        super().__init__(msg)
+        self.status = status
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t, name, dtype, shape, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _prepare(x, dt, A, B, C_, Dskip, block, z, dt_softplus):
+    if not isinstance(x, torch.Tensor) or x.dim() != 3:
+        raise ValueError("x must be a [batch, L, D] tensor")
+    _check_device(x.device)
+    Bt, L, D = x.shape
+    N = B.shape[-1] if isinstance(B, torch.Tensor) and B.dim() == 3 else -1
+    io = x.dtype
+    if io not in (torch.float32, torch.bfloat16):
+        raise TypeError("io dtype must be float32 or bfloat16")
+    dev = x.device
+    _need(x, "x", io, (Bt, L, D), dev)
+    _need(dt, "dt", io, (Bt, L, D), dev)
+    _need(B, "B", io, (Bt, L, N), dev)
+    _need(C_, "C", io, (Bt, L, N), dev)
+    _need(A, "A", torch.float32, (D, N), dev)
+    _need(Dskip, "Dskip", torch.float32, (D,), dev)
+    if z is not None:
+        _need(z, "z", io, (Bt, L, D), dev)
+    dims = Dims(Bt, L, D, N, int(block), BF16 if io == torch.bfloat16 else F32, 1 if dt_softplus else 0)
+    ins = Inputs(_ptr(x), _ptr(dt), _ptr(B), _ptr(C_), _ptr(z), _ptr(A), _ptr(Dskip))
+    return dims, ins, (Bt, L, D, N), io, dev
+
+
+def _check_device(device):
+    if device.type != "cuda":
+        raise ValueError("bdscan runs on CUDA tensors only")
+
+
+def _stream(dev):
+    return torch.cuda.current_stream(dev).cuda_stream
+
+
+def _check(rc, where):
+    if rc != 0:
+        raise BdscanError(rc, where)
+
+
+def train_blocks(x, dt, A, B, C, Dskip, block, z=None, h0=None, dt_softplus=True,
+                 y=None, boundary=None, h_out=None, want_boundary=False, want_h_out=False):
+    """Full-block pass over every block of every sequence: returns (y, boundary, h_out).
+
+    boundary / h_out are returned when passed in or requested, else None.
+    """
+    dims, ins, (Bt, L, D, N), io, dev = _prepare(x, dt, A, B, C, Dskip, block, z, dt_softplus)
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (Bt, D, N), dev)
+    y = torch.empty((Bt, L, D), dtype=io, device=dev) if y is None else y
+    _need(y, "y", io, (Bt, L, D), dev)
+    if boundary is None and want_boundary:
+        boundary = torch.empty((Bt, L // max(int(block), 1), D, N), dtype=torch.float32, device=dev)
+    if boundary is not None:
+        _need(boundary, "boundary", torch.float32, (Bt, L // int(block), D, N), dev)
+    if h_out is None and want_h_out:
+        h_out = torch.empty((Bt, D, N), dtype=torch.float32, device=dev)
+    if h_out is not None:
+        _need(h_out, "h_out", torch.float32, (Bt, D, N), dev)
+    rc = _lib.bdscan_train_blocks(ct.byref(dims), ct.byref(ins), _ptr(h0), _ptr(y), _ptr(boundary),
+                                  _ptr(h_out), _stream(dev))
+    _check(rc, "bdscan_train_blocks")
+    return y, boundary, h_out
+
+
+def prefill(x, dt, A, B, C, Dskip, block, z=None, h0=None, dt_softplus=True,
+            want_y=True, y=None, h_out=None, boundary=None, want_boundary=False):
+    """Forward-only scan of a clean context: returns (y or None, h_out, boundary or None)."""
+    dims, ins, (Bt, L, D, N), io, dev = _prepare(x, dt, A, B, C, Dskip, block, z, dt_softplus)
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (Bt, D, N), dev)
+    if y is None and want_y:
+        y = torch.empty((Bt, L, D), dtype=io, device=dev)
+    if y is not None:
+        _need(y, "y", io, (Bt, L, D), dev)
+    h_out = torch.empty((Bt, D, N), dtype=torch.float32, device=dev) if h_out is None else h_out
+    _need(h_out, "h_out", torch.float32, (Bt, D, N), dev)
+    if boundary is None and want_boundary:
+        boundary = torch.empty((Bt, L // int(block), D, N), dtype=torch.float32, device=dev)
+    if boundary is not None:
+        _need(boundary, "boundary", torch.float32, (Bt, L // int(block), D, N), dev)
+    rc = _lib.bdscan_prefill(ct.byref(dims), ct.byref(ins), _ptr(h0), _ptr(y), _ptr(h_out),
+                             _ptr(boundary), _stream(dev))
+    _check(rc, "bdscan_prefill")
+    return y, h_out, boundary
+
+
+def block_step(x, dt, A, B, C, Dskip, h_cache, z=None, dt_softplus=True, y=None):
+    """One denoising step of the active block (L == block): returns y. h_cache is read only."""
+    block = x.shape[1]
+    dims, ins, (Bt, L, D, N), io, dev = _prepare(x, dt, A, B, C, Dskip, block, z, dt_softplus)
+    _need(h_cache, "h_cache", torch.float32, (Bt, D, N), dev)
+    y = torch.empty((Bt, L, D), dtype=io, device=dev) if y is None else y
+    _need(y, "y", io, (Bt, L, D), dev)
+    rc = _lib.bdscan_block_step(ct.byref(dims), ct.byref(ins), _ptr(h_cache), _ptr(y), _stream(dev))
+    _check(rc, "bdscan_block_step")
+    return y
+
+
+def commit_block(x, dt, A, B, C, Dskip, h_cache, z=None, dt_softplus=True, want_y=False, y=None):
+    """Commit a clean block (L == block): advances h_cache in place; returns y or None."""
+    block = x.shape[1]
+    dims, ins, (Bt, L, D, N), io, dev = _prepare(x, dt, A, B, C, Dskip, block, z, dt_softplus)
+    _need(h_cache, "h_cache", torch.float32, (Bt, D, N), dev)
+    if y is None and want_y:
+        y = torch.empty((Bt, L, D), dtype=io, device=dev)
+    if y is not None:
+        _need(y, "y", io, (Bt, L, D), dev)
+    rc = _lib.bdscan_commit_block(ct.byref(dims), ct.byref(ins), _ptr(h_cache), _ptr(y), _stream(dev))
+    _check(rc, "bdscan_commit_block")
+    return y
+
+
+def raw_library():
+    """The loaded ctypes library (for tests that call the C ABI directly)."""
+    return _lib

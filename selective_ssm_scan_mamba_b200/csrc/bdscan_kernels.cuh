@@ -1,0 +1,474 @@
+// The block-confined bidirectional selective-scan kernel family (sm_100a).
+//
+// Method: "Training Hybrid Block Diffusion Language Models with Partial
+// Bidirectionality" (arXiv 2607.02805), abstract and gist.science technical
+// summary ("Methodik"): a causal forward Mamba scan whose block-end states are
+// the exact cache, plus a reverse scan confined to each denoising block.
+//
+// Work decomposition
+//   grid   = (ceil(D / 32), batch). A CTA owns 32 channels of one sequence and
+//            walks all L tokens in order; the forward state never leaves
+//            registers.
+//   warps  = lane = channel, warp = state group: warp w holds states
+//            [w*NPT, (w+1)*NPT) of all 32 channels (W = N / NPT warps). A
+//            warp's B and C reads are then the same address in every lane
+//            (one shared-memory wavefront), and delta is read once per lane.
+//   tiles  = T tokens (16, or 32 for 32-token blocks). x/dt/z [T x 32] and B/C
+//            [T x N] arrive in shared memory by 16-byte cp.async through a ring
+//            of stages; the CTA then computes delta = softplus(dt), delta*x and
+//            the fp32 B/C once per element.
+//   spans  = each span (a block of up to 32 tokens, or 16 tokens) runs in three
+//            phases so a warp always has independent work in flight:
+//            (A) decays a = 2^(delta A log2 e) (one MUFU.EX2 per token, channel
+//                and state) and inputs b = delta x B for every token of the
+//                span -- no dependence between tokens;
+//            (B) the forward chain h = a h + b with its readout C.h;
+//            (C) the block-confined reverse chain g = a g + b from the kept a
+//                (and b), so the reverse costs no second exp.
+//            Recurrences and readouts use packed fp32x2 FMA (two states per
+//            instruction).
+//   readout= each warp's partial sums C.(h + g) go through a padded shared-memory
+//            buffer; warp w then sums the W partials of its share of the tile's
+//            tokens, adds the skip term, applies the gate and stores y.
+//   long   = blocks longer than 32 tokens: per block, a reverse sweep over its
+//            tiles from last to first (carrying g) whose readout is staged in
+//            shared memory, then a forward sweep that adds it (two exps per
+//            element).
+#pragma once
+
+#include "bdscan_device.cuh"
+
+namespace bdk {
+
+constexpr int kCh = 32;                  // channels per CTA (one per lane)
+constexpr int kLongSmemMax = 96 * 1024;  // y_rev staging limit of the long-block path
+
+enum Mode { kForwardOnly = 0, kFused = 1, kLong = 2 };
+
+struct ScanArgs {
+    const void *x, *dt, *B, *C, *z;
+    const float *A, *Dskip, *h0;
+    void *y;
+    float *h_out, *boundary;
+    int64_t L, D;
+    int32_t K, dt_softplus;
+};
+
+// States per lane: 4 where a block's decays are kept for the reverse scan;
+// the forward-only N = 16 variant spreads one state per warp (16 warps) for
+// parallelism on single-sequence prefills.
+template <int N, int MODE>
+struct Npt {
+    static constexpr int value = (MODE == kForwardOnly && N == 16) ? 1 : 4;
+};
+
+template <int N, int MODE, int KC>
+struct Cfg {
+    static constexpr int NPT = Npt<N, MODE>::value;
+    static constexpr int W = N / NPT;                 // warps per CTA (state groups)
+    static constexpr int THREADS = 32 * W;
+    static constexpr int T = (MODE == kFused && (KC == 0 || KC > 16)) ? 32 : 16;   // tokens per tile
+    static constexpr int S = T == 16 ? 4 : 3;                                    // cp.async ring depth
+    static constexpr int SPAN = MODE == kFused ? (KC > 0 ? KC : T) : 16;
+    static constexpr bool KEEP_B = SPAN <= 16 && N == 16;                        // keep b for phase C
+    static constexpr int PER = T / W > 0 ? T / W : 1;                            // readout tokens per warp
+    // registers: the four N = 16 state-group warps of a CTA sit on the SM's four
+    // sub-partitions, so 3 resident CTAs = 3 warps per sub-partition (<= 168
+    // registers), enough for a 12288-channel batch in one wave on 148 SMs.
+    static constexpr int MINB = THREADS >= 512 ? 1 : (T == 16 ? 3 : 2);
+    static_assert(N % NPT == 0 && W <= 32, "state split");
+};
+
+// Shared-memory carve-up (bytes; every offset is a multiple of 16).
+template <class IO, int N, int MODE, int KC>
+struct Layout {
+    using CF = Cfg<N, MODE, KC>;
+    static constexpr int T = CF::T, S = CF::S, W = CF::W;
+    static constexpr int RP = T + 4;                       // padded row of the readout buffer
+    static constexpr int xb = T * kCh * (int)sizeof(IO);   // one x / dt / z tile
+    static constexpr int bb = T * N * (int)sizeof(IO);     // one B / C tile
+    static constexpr int stage = 3 * xb + 2 * bb;
+    static constexpr int dd = S * stage;                   // float2 (delta, delta*x)   [T][32]
+    static constexpr int bf = dd + T * kCh * 8;            // float B                  [T][N]
+    static constexpr int cf = bf + T * N * 4;              // float C                  [T][N]
+    static constexpr int red = cf + T * N * 4;             // float partial readouts   [W][32][RP]
+    static constexpr int yrev = red + W * kCh * RP * 4;    // float reverse readout    [K][32] (long)
+    static constexpr int base_bytes = yrev;
+    static_assert(xb % 16 == 0 && bb % 16 == 0 && (RP * 4) % 16 == 0, "16-byte rows");
+};
+
+// ---- per-lane arithmetic on NPT states (NPT = 1, 2 or 4) -----------------------
+// Every mode runs these same instructions, so the forward state is
+// bit-identical whichever kernel variant computes it (packed and scalar fp32
+// operations round identically).
+
+// decays a[n] = 2^(delta * A'[n]) (A' = A log2 e) and inputs b[n] = (delta x) B[n]
+template <int NPT>
+__device__ __forceinline__ void decay_input(const float (&al)[NPT], float2 dv, const float *Bn, float (&a)[NPT],
+                                            float (&bq)[NPT]) {
+    if constexpr (NPT == 1) {
+        a[0] = ex2_approx(__fmul_rn(dv.x, al[0]));
+        bq[0] = __fmul_rn(dv.y, Bn[0]);
+    } else {
+        const float2 d2 = make_float2(dv.x, dv.x), x2 = make_float2(dv.y, dv.y);
+#pragma unroll
+        for (int p = 0; p < NPT / 2; ++p) {
+            const float2 e = __fmul2_rn(d2, make_float2(al[2 * p], al[2 * p + 1]));
+            a[2 * p] = ex2_approx(e.x);
+            a[2 * p + 1] = ex2_approx(e.y);
+            const float2 bb = __fmul2_rn(x2, make_float2(Bn[2 * p], Bn[2 * p + 1]));
+            bq[2 * p] = bb.x;
+            bq[2 * p + 1] = bb.y;
+        }
+    }
+}
+
+// inputs only: b[n] = (delta x) B[n]  (the same instructions as in decay_input)
+template <int NPT>
+__device__ __forceinline__ void input_only(float dx, const float *Bn, float (&bq)[NPT]) {
+    if constexpr (NPT == 1) {
+        bq[0] = __fmul_rn(dx, Bn[0]);
+    } else {
+        const float2 x2 = make_float2(dx, dx);
+#pragma unroll
+        for (int p = 0; p < NPT / 2; ++p) {
+            const float2 bb = __fmul2_rn(x2, make_float2(Bn[2 * p], Bn[2 * p + 1]));
+            bq[2 * p] = bb.x;
+            bq[2 * p + 1] = bb.y;
+        }
+    }
+}
+
+// one recurrence step s = a s + b; returns the lane's partial sum_n C[n] s[n]
+template <int NPT>
+__device__ __forceinline__ float scan_step(float (&st)[NPT], const float (&a)[NPT], const float (&bq)[NPT],
+                                           const float *Cn) {
+    if constexpr (NPT == 1) {
+        st[0] = __fmaf_rn(a[0], st[0], bq[0]);
+        return __fmul_rn(Cn[0], st[0]);
+    } else {
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int p = 0; p < NPT / 2; ++p) {
+            const float2 s2 = __ffma2_rn(make_float2(a[2 * p], a[2 * p + 1]), make_float2(st[2 * p], st[2 * p + 1]),
+                                         make_float2(bq[2 * p], bq[2 * p + 1]));
+            st[2 * p] = s2.x;
+            st[2 * p + 1] = s2.y;
+            const float2 c2 = make_float2(Cn[2 * p], Cn[2 * p + 1]);
+            acc = p == 0 ? __fmul2_rn(c2, s2) : __ffma2_rn(c2, s2, acc);
+        }
+        return __fadd_rn(acc.x, acc.y);
+    }
+}
+
+// Copy tokens [t0, t0 + tlen) of one CTA's tile into a ring stage; rows past
+// tlen and channels past D are zero-filled without reading global memory.
+template <class IO, int N, int T, int NT>
+__device__ __forceinline__ void stage_tile(char *st, const ScanArgs &a, int64_t b, int64_t d0, int64_t t0,
+                                           int tlen, bool gated) {
+    constexpr int EPC = 16 / (int)sizeof(IO);   // elements per 16-byte chunk
+    constexpr int XC = kCh / EPC;               // chunks per x row
+    constexpr int BC = N / EPC;                 // chunks per B row
+    IO *xs = reinterpret_cast<IO *>(st);
+    IO *dts = xs + T * kCh;
+    IO *zs = dts + T * kCh;
+    IO *Bs = zs + T * kCh;
+    IO *Cs = Bs + T * N;
+    const int64_t row0 = b * a.L + t0;   // first token row of the tile
+    for (int e = threadIdx.x; e < T * XC; e += NT) {
+        const int t = e / XC, ch = e % XC;
+        const int64_t d = d0 + (int64_t)ch * EPC;
+        const bool ok = t < tlen && d < a.D;
+        const int64_t off = ok ? ((row0 + t) * a.D + d) : 0;
+        const int so = t * kCh + ch * EPC;
+        cp_async16(xs + so, static_cast<const IO *>(a.x) + off, ok);
+        cp_async16(dts + so, static_cast<const IO *>(a.dt) + off, ok);
+        if (gated) cp_async16(zs + so, static_cast<const IO *>(a.z) + off, ok);
+    }
+    for (int e = threadIdx.x; e < T * BC; e += NT) {
+        const int t = e / BC, ch = e % BC;
+        const bool ok = t < tlen;
+        const int64_t off = ok ? ((row0 + t) * N + (int64_t)ch * EPC) : 0;
+        const int so = t * N + ch * EPC;
+        cp_async16(Bs + so, static_cast<const IO *>(a.B) + off, ok);
+        cp_async16(Cs + so, static_cast<const IO *>(a.C) + off, ok);
+    }
+}
+
+// One CTA = one (batch row, 32-channel tile). MODE selects forward-only, fused
+// (block <= 32; KC = compile-time block length, or 0 for a runtime one), or
+// the long-block two-sweep path.
+template <class IO, int N, int MODE, int KC>
+__global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::MINB)
+    bdscan_kernel(const ScanArgs a) {
+    using CF = Cfg<N, MODE, KC>;
+    using LY = Layout<IO, N, MODE, KC>;
+    constexpr int NPT = CF::NPT, W = CF::W, NT = CF::THREADS, T = CF::T, S = CF::S, SPAN = CF::SPAN;
+    constexpr int RP = LY::RP, PER = CF::PER;
+    constexpr bool KEEP_B = CF::KEEP_B;
+    static_assert(T % SPAN == 0, "spans tile the tile");
+
+    extern __shared__ __align__(16) char smem[];
+    float2 *dd = reinterpret_cast<float2 *>(smem + LY::dd);
+    float *Bf = reinterpret_cast<float *>(smem + LY::bf);
+    float *Cf = reinterpret_cast<float *>(smem + LY::cf);
+    float *red = reinterpret_cast<float *>(smem + LY::red);
+    float *yrev = reinterpret_cast<float *>(smem + LY::yrev);
+
+    const int tid = threadIdx.x, c = tid & 31, warp = tid >> 5;
+    const int n0 = warp * NPT;                 // this warp's states
+    const int64_t b = blockIdx.y;
+    const int64_t d0 = (int64_t)blockIdx.x * kCh;
+    const int64_t d = d0 + c;
+    const bool dvalid = d < a.D;
+    const int64_t L = a.L, K = a.K;
+    const bool gated = a.z != nullptr;
+    const bool want_y = a.y != nullptr;
+    const float dskip = dvalid ? a.Dskip[d] : 0.f;
+    const float dfac = MODE == kForwardOnly ? dskip : __fmul_rn(2.f, dskip);
+
+    // per-lane constants: A[d, n] * log2(e) and the initial state
+    float al[NPT], h[NPT], gcar[NPT];
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) {
+        al[j] = dvalid ? __fmul_rn(a.A[d * N + n0 + j], kLog2e) : 0.f;
+        h[j] = (dvalid && a.h0) ? a.h0[(b * a.D + d) * N + n0 + j] : 0.f;
+        gcar[j] = 0.f;   // reverse carry across tiles (long path)
+    }
+
+    // ---- tile schedule ------------------------------------------------------
+    // forward-only / fused: step s covers tokens [s*TE, min((s+1)*TE, L)).
+    // long: per block j, nt reverse steps (tiles nt-1 .. 0) then nt forward steps.
+    const int TE = (MODE == kFused && KC == 0) ? (int)((T / K) * K) : T;
+    const int64_t nt_blk = (MODE == kLong) ? (K + T - 1) / T : 1;
+    const int64_t nsteps = (MODE == kLong) ? (L / K) * 2 * nt_blk : (L + TE - 1) / TE;
+    auto tile_of = [&](int64_t s, int64_t &t0, int &tlen, bool &rev, bool &first_rev) {
+        if (MODE == kLong) {
+            const int64_t j = s / (2 * nt_blk), r = s % (2 * nt_blk);
+            rev = r < nt_blk;
+            const int64_t i = rev ? nt_blk - 1 - r : r - nt_blk;
+            first_rev = rev && r == 0;
+            t0 = j * K + i * T;
+            const int64_t rem = (j + 1) * K - t0;
+            tlen = (int)(rem < T ? rem : T);
+        } else {
+            rev = false;
+            first_rev = false;
+            t0 = s * TE;
+            const int64_t rem = L - t0;
+            tlen = (int)(rem < TE ? rem : TE);
+        }
+    };
+    auto issue = [&](int64_t s) {
+        if (s < nsteps) {
+            int64_t t0; int tlen; bool rv, fr;
+            tile_of(s, t0, tlen, rv, fr);
+            stage_tile<IO, N, T, NT>(smem + (s % S) * LY::stage, a, b, d0, t0, tlen, gated);
+        }
+        cp_async_commit();
+    };
+
+    const int64_t nblk = L / K;
+    float *bnd_ptr = (a.boundary && dvalid) ? a.boundary + (b * nblk * a.D + d) * N + n0 : nullptr;
+    const int64_t bnd_stride = a.D * N;   // between consecutive block ends
+    auto write_boundary = [&](int64_t tok_end) {   // state after token tok_end (a block end)
+        if (bnd_ptr) {
+            float *p = bnd_ptr + ((tok_end + 1) / K - 1) * bnd_stride;
+            if constexpr (NPT == 4) *reinterpret_cast<float4 *>(p) = make_float4(h[0], h[1], h[2], h[3]);
+            else if constexpr (NPT == 2) *reinterpret_cast<float2 *>(p) = make_float2(h[0], h[1]);
+            else p[0] = h[0];
+        }
+    };
+
+    const float2 *ddc = dd + c;    // row t: ddc[t * 32]
+    const float *Bw = Bf + n0;     // row t: Bw + t * N   (same address in every lane)
+    const float *Cw = Cf + n0;
+
+#pragma unroll 1
+    for (int s = 0; s < S - 1; ++s) issue(s);
+
+#pragma unroll 1
+    for (int64_t s = 0; s < nsteps; ++s) {
+        int64_t t0; int tlen; bool rev, first_rev;
+        tile_of(s, t0, tlen, rev, first_rev);
+        cp_async_wait<S - 2>();
+        __syncthreads();   // stage s landed for every thread; step s-1 is fully done
+        issue(s + S - 1);
+        const char *st = smem + (s % S) * LY::stage;
+        const IO *xs = reinterpret_cast<const IO *>(st);
+        const IO *dts = xs + T * kCh;
+        const IO *zs = dts + T * kCh;
+
+        // ---- per-element preprocessing, once per CTA ----------------------------
+        {
+            const IO *Bs = zs + T * kCh;
+            const IO *Cs = Bs + T * N;
+            for (int e = tid; e < T * kCh; e += NT) {
+                const float xv = to_f32(xs[e]);
+                const float dr = to_f32(dts[e]);
+                const float dl = a.dt_softplus ? softplus_f32(dr) : dr;
+                dd[e] = make_float2(dl, __fmul_rn(dl, xv));
+            }
+            constexpr int EPC = 16 / (int)sizeof(IO);
+            for (int e = tid; e < T * N / EPC; e += NT) {
+                widen16(Bs + e * EPC, Bf + e * EPC);
+                widen16(Cs + e * EPC, Cf + e * EPC);
+            }
+        }
+        __syncthreads();
+
+        // ---- the scan over this tile --------------------------------------------
+        float yp[T];
+        uint32_t endmask = 0;   // block ends inside the tile (runtime-K and forward-only)
+        if (MODE == kForwardOnly || (MODE == kFused && KC == 0)) {
+            for (int64_t e = K - 1 - (t0 % K); e < tlen; e += K) endmask |= 1u << e;
+        } else if (MODE == kLong) {
+            if (!rev && (t0 + tlen) % K == 0) endmask = 1u << (tlen - 1);
+        }
+
+        if (MODE == kLong && rev) {   // reverse sweep tile of a long block: decays, then the chain
+            float at[T][NPT];
+#pragma unroll
+            for (int t = 0; t < T; ++t) {
+                float bq[NPT];
+                decay_input<NPT>(al, t < tlen ? ddc[t * kCh] : make_float2(0.f, 0.f), Bw + t * N, at[t], bq);
+            }
+            if (first_rev) {
+#pragma unroll
+                for (int j = 0; j < NPT; ++j) gcar[j] = 0.f;
+            }
+#pragma unroll
+            for (int t = T - 1; t >= 0; --t) {
+                float acc = 0.f;
+                if (t < tlen) {
+                    float bq[NPT];
+                    input_only<NPT>(ddc[t * kCh].y, Bw + t * N, bq);
+                    acc = scan_step<NPT>(gcar, at[t], bq, Cw + t * N);
+                }
+                yp[t] = acc;
+            }
+        } else {
+            constexpr bool REV = MODE == kFused;
+            constexpr int NB = KEEP_B ? SPAN : 1;
+#pragma unroll
+            for (int sp = 0; sp < T / SPAN; ++sp) {
+                const int s0 = sp * SPAN;
+                const bool whole = s0 + SPAN <= tlen;   // all span tokens valid (else a ragged tail)
+                float at[SPAN][NPT];
+                float bt[NB][NPT];
+#pragma unroll
+                for (int i = 0; i < SPAN; ++i) {   // (A)
+                    const bool ok = whole || s0 + i < tlen;
+                    float bq[NPT];
+                    decay_input<NPT>(al, ok ? ddc[(s0 + i) * kCh] : make_float2(0.f, 0.f), Bw + (s0 + i) * N,
+                                     at[i], bq);
+                    if (KEEP_B) {
+#pragma unroll
+                        for (int j = 0; j < NPT; ++j) bt[KEEP_B ? i : 0][j] = bq[j];
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < SPAN; ++i) {   // (B)
+                    const int t = s0 + i;
+                    float acc = 0.f;
+                    if (whole || t < tlen) {
+                        float bq[NPT];
+                        if (KEEP_B) {
+#pragma unroll
+                            for (int j = 0; j < NPT; ++j) bq[j] = bt[KEEP_B ? i : 0][j];
+                        } else {
+                            input_only<NPT>(ddc[t * kCh].y, Bw + t * N, bq);
+                        }
+                        acc = scan_step<NPT>(h, at[i], bq, Cw + t * N);
+                        if (MODE == kFused && KC > 0 ? (i == SPAN - 1) : ((endmask >> t) & 1u)) write_boundary(t0 + t);
+                    }
+                    yp[t] = acc;
+                }
+                if (REV) {
+                    float gs[NPT];
+#pragma unroll
+                    for (int j = 0; j < NPT; ++j) gs[j] = 0.f;
+#pragma unroll
+                    for (int i = SPAN - 1; i >= 0; --i) {   // (C)
+                        const int t = s0 + i;
+                        if (whole || t < tlen) {
+                            if (KC == 0 && ((endmask >> t) & 1u)) {
+#pragma unroll
+                                for (int j = 0; j < NPT; ++j) gs[j] = 0.f;
+                            }
+                            float bq[NPT];
+                            if (KEEP_B) {
+#pragma unroll
+                                for (int j = 0; j < NPT; ++j) bq[j] = bt[KEEP_B ? i : 0][j];
+                            } else {
+                                input_only<NPT>(ddc[t * kCh].y, Bw + t * N, bq);
+                            }
+                            yp[t] = __fadd_rn(yp[t], scan_step<NPT>(gs, at[i], bq, Cw + t * N));
+                        }
+                    }
+                }
+            }
+        }
+
+        // ---- readout: the W state-group partials of every (token, channel) -------
+        {
+            float *rrow = red + (warp * kCh + c) * RP;   // this warp's partials for channel c
+#pragma unroll
+            for (int q = 0; q < T / 4; ++q)
+                *reinterpret_cast<float4 *>(rrow + 4 * q) =
+                    make_float4(yp[4 * q], yp[4 * q + 1], yp[4 * q + 2], yp[4 * q + 3]);
+        }
+        __syncthreads();
+        // warp w finishes tokens [w*PER, (w+1)*PER) of the tile
+        if (warp * PER < T) {
+            float ysum[PER];
+#pragma unroll
+            for (int i = 0; i < PER; ++i) ysum[i] = 0.f;
+#pragma unroll
+            for (int gg = 0; gg < W; ++gg) {
+                const float *rrow = red + (gg * kCh + c) * RP + warp * PER;
+                if constexpr (PER % 4 == 0) {
+#pragma unroll
+                    for (int q = 0; q < PER / 4; ++q) {
+                        const float4 v = *reinterpret_cast<const float4 *>(rrow + 4 * q);
+                        ysum[4 * q] = __fadd_rn(ysum[4 * q], v.x);
+                        ysum[4 * q + 1] = __fadd_rn(ysum[4 * q + 1], v.y);
+                        ysum[4 * q + 2] = __fadd_rn(ysum[4 * q + 2], v.z);
+                        ysum[4 * q + 3] = __fadd_rn(ysum[4 * q + 3], v.w);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < PER; ++i) ysum[i] = __fadd_rn(ysum[i], rrow[i]);
+                }
+            }
+            IO *gy = want_y ? static_cast<IO *>(a.y) + (b * L + t0) * a.D + d : nullptr;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int t = warp * PER + i;
+                if (t < tlen) {
+                    const int yr = (int)(t0 - (t0 / K) * K) + t;   // token within its block (long path)
+                    if (MODE == kLong && rev) {
+                        yrev[yr * kCh + c] = ysum[i];
+                    } else if (want_y && dvalid) {
+                        float v = ysum[i];
+                        if (MODE == kLong) v = __fadd_rn(v, yrev[yr * kCh + c]);
+                        v = __fmaf_rn(dfac, to_f32(xs[t * kCh + c]), v);
+                        if (gated) v = __fmul_rn(v, silu_f32(to_f32(zs[t * kCh + c])));
+                        IO o;
+                        from_f32(v, o);
+                        gy[(int64_t)t * a.D] = o;
+                    }
+                }
+            }
+        }
+    }
+    cp_async_wait<0>();
+
+    if (a.h_out && dvalid) {
+        float *p = a.h_out + (b * a.D + d) * N + n0;
+#pragma unroll
+        for (int j = 0; j < NPT; ++j) p[j] = h[j];
+    }
+}
+
+}  // namespace bdk

@@ -26,6 +26,9 @@ and returned as their raw ``uint16`` bit patterns.
 from __future__ import annotations
 
 import dataclasses
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 CHUNK = 4096  # tokens per independently seeded chunk
@@ -36,11 +39,16 @@ _STREAM_IDS = {"seq": 0, "context": 1, "noisy": 2, "clean": 3, "layer": 4}
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
-    """Round fp32 to bf16 (round to nearest, ties to even); returns uint16 bits."""
-    a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return rounded.astype(np.uint16)
+    """Round finite fp32 to bf16 (round to nearest, ties to even); returns uint16 bits.
+
+    The 32-bit sum cannot wrap for finite inputs: the largest finite pattern
+    0xFF7FFFFF plus 0x8000 stays below 2**32."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    r = (u >> 16) & np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += u
+    r >>= 16
+    return r.astype(np.uint16)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -59,20 +67,18 @@ def _stream_key(stream) -> tuple:
     return (_STREAM_IDS[name], *[int(r) for r in rest])
 
 
-def _draw_rows(seed, array, stream, b, t0, t1, width, mean, std):
-    """fp32 draws for tokens [t0, t1) of batch row b, assembled from fixed chunks."""
-    out = np.empty((t1 - t0, width), dtype=np.float32)
-    c0, c1 = t0 // CHUNK, (t1 - 1) // CHUNK if t1 > t0 else t0 // CHUNK - 1
-    for c in range(c0, c1 + 1):
-        g = _rng(seed, _ARRAY_IDS[array], *_stream_key(stream), b, c)
-        blk = g.standard_normal((CHUNK, width), dtype=np.float32)
-        if std != 1.0:
-            blk *= np.float32(std)
-        if mean != 0.0:
-            blk += np.float32(mean)
-        lo, hi = max(t0, c * CHUNK), min(t1, (c + 1) * CHUNK)
-        out[lo - t0:hi - t0] = blk[lo - c * CHUNK:hi - c * CHUNK]
-    return out
+def _draw_chunk(seed, array, stream, b, c, width, mean, std):
+    g = _rng(seed, _ARRAY_IDS[array], *_stream_key(stream), b, c)
+    blk = g.standard_normal((CHUNK, width), dtype=np.float32)
+    if std != 1.0:
+        blk *= np.float32(std)
+    if mean != 0.0:
+        blk += np.float32(mean)
+    return blk
+
+
+def _chunk_range(t0, t1):
+    return range(t0 // CHUNK, (t1 - 1) // CHUNK + 1) if t1 > t0 else range(0)
 
 
 def _cast(a32: np.ndarray, io: str) -> np.ndarray:
@@ -92,19 +98,31 @@ def make_sequence(seed: int, batch: int, L: int, D: int, N: int, io: str,
     (B and C are shared by all channels and always returned whole).
     """
     t1 = t0 + L
-    out = {k: [] for k in (("x", "dt", "B", "C", "z") if gated else ("x", "dt", "B", "C"))}
-    for b in range(batch):
-        for name, width, mean, std in (("x", D, 0.0, 1.0), ("dt", D, -2.0, 0.5),
-                                       ("B", N, 0.0, 1.0 / np.sqrt(N)),
-                                       ("C", N, 0.0, 1.0 / np.sqrt(N)),
-                                       ("z", D, 0.0, 1.0)):
-            if name not in out:
-                continue
-            rows = _draw_rows(seed, name, stream, b, t0, t1, width, mean, std)
-            if channels is not None and name in ("x", "dt", "z"):
-                rows = rows[:, channels]
-            out[name].append(_cast(rows, io))
-    return {k: np.ascontiguousarray(np.stack(v)) for k, v in out.items()}
+    specs = [("x", D, 0.0, 1.0), ("dt", D, -2.0, 0.5), ("B", N, 0.0, 1.0 / np.sqrt(N)),
+             ("C", N, 0.0, 1.0 / np.sqrt(N))] + ([("z", D, 0.0, 1.0)] if gated else [])
+    store = np.uint16 if io == "bf16" else np.float32
+    res = {}
+    for name, width, _, _ in specs:
+        w_out = len(channels) if (channels is not None and name in ("x", "dt", "z")) else width
+        res[name] = np.empty((batch, L, w_out), dtype=store)
+
+    def job(name, width, mean, std, b, c):
+        blk = _draw_chunk(seed, name, stream, b, c, width, mean, std)
+        lo, hi = max(t0, c * CHUNK), min(t1, (c + 1) * CHUNK)
+        part = blk[lo - c * CHUNK:hi - c * CHUNK]
+        if channels is not None and name in ("x", "dt", "z"):
+            part = part[:, channels]
+        res[name][b, lo - t0:hi - t0] = _cast(part, io)
+
+    jobs = [(name, width, mean, std, b, c) for name, width, mean, std in specs
+            for b in range(batch) for c in _chunk_range(t0, t1)]
+    if len(jobs) > 2 and batch * L * D >= (1 << 22):
+        with ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 1)) as ex:
+            list(ex.map(lambda j: job(*j), jobs))
+    else:
+        for j in jobs:
+            job(*j)
+    return res
 
 
 def make_params(seed: int, D: int, N: int, layer: int = 0) -> dict:

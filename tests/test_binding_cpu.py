@@ -1,0 +1,95 @@
+"""The Python binding's marshalling, driven on CPU tensors against a fake
+library that records each call (no GPU, no kernel launch)."""
+import ctypes as ct
+
+import pytest
+import torch
+
+from selective_ssm_scan_mamba_b200 import bdscan
+
+
+class FakeLib:
+    def __init__(self, rc=0):
+        self.calls = []
+        self.rc = rc
+
+    def _rec(self, name):
+        def f(*args):
+            self.calls.append((name, args))
+            return self.rc
+        return f
+
+    def __getattr__(self, name):
+        if name.startswith("bdscan_"):
+            return self._rec(name)
+        raise AttributeError(name)
+
+
+@pytest.fixture
+def fake(monkeypatch):
+    lib = FakeLib()
+    monkeypatch.setattr(bdscan, "_lib", lib)
+    monkeypatch.setattr(bdscan, "_check_device", lambda d: None)
+    monkeypatch.setattr(bdscan, "_stream", lambda d: 1234)
+    return lib
+
+
+def tensors(Bt=2, L=32, D=64, N=16, io=torch.bfloat16):
+    return dict(x=torch.zeros(Bt, L, D, dtype=io), dt=torch.zeros(Bt, L, D, dtype=io),
+                A=torch.zeros(D, N), B=torch.zeros(Bt, L, N, dtype=io), C=torch.zeros(Bt, L, N, dtype=io),
+                Dskip=torch.zeros(D))
+
+
+def _dims(arg):
+    return ct.cast(arg, ct.POINTER(bdscan.Dims)).contents if not isinstance(arg, bdscan.Dims) else arg
+
+
+def test_train_blocks_marshalling(fake):
+    t = tensors()
+    y, bnd, h = bdscan.train_blocks(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], 16,
+                                    want_boundary=True, want_h_out=True)
+    name, args = fake.calls[-1]
+    assert name == "bdscan_train_blocks"
+    assert y.shape == (2, 32, 64) and y.dtype == torch.bfloat16
+    assert bnd.shape == (2, 2, 64, 16) and h.shape == (2, 64, 16)
+    assert args[2] is None and args[3] == y.data_ptr() and args[4] == bnd.data_ptr() and args[5] == h.data_ptr()
+    assert args[6] == 1234
+
+
+def test_each_entry_point_reaches_the_library(fake):
+    t = tensors(L=16)
+    cache = torch.zeros(2, 64, 16)
+    bdscan.prefill(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], 16)
+    bdscan.block_step(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], cache)
+    bdscan.commit_block(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], cache, want_y=True)
+    assert [c[0] for c in fake.calls] == ["bdscan_prefill", "bdscan_block_step", "bdscan_commit_block"]
+    assert fake.calls[1][1][2] == cache.data_ptr() and fake.calls[2][1][2] == cache.data_ptr()
+
+
+def test_status_becomes_exception(monkeypatch):
+    lib = FakeLib(rc=2)
+    lib.bdscan_status_string = lambda s: b"BDSCAN_ERR_UNSUPPORTED"
+    monkeypatch.setattr(bdscan, "_lib", lib)
+    monkeypatch.setattr(bdscan, "_check_device", lambda d: None)
+    monkeypatch.setattr(bdscan, "_stream", lambda d: 0)
+    t = tensors()
+    with pytest.raises(bdscan.BdscanError, match="UNSUPPORTED"):
+        bdscan.train_blocks(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], 16)
+
+
+def test_shape_dtype_and_layout_checks(fake):
+    t = tensors()
+    with pytest.raises(TypeError):
+        bdscan.train_blocks(t["x"].float(), t["dt"], t["A"], t["B"], t["C"], t["Dskip"], 16)
+    with pytest.raises(ValueError):
+        bdscan.train_blocks(t["x"], t["dt"], t["A"][:32], t["B"], t["C"], t["Dskip"], 16)
+    with pytest.raises(ValueError):
+        bdscan.train_blocks(t["x"].transpose(1, 2).contiguous().transpose(1, 2), t["dt"], t["A"], t["B"],
+                            t["C"], t["Dskip"], 16)
+    assert not fake.calls
+
+
+def test_cpu_tensors_are_refused_without_fallback():
+    t = tensors()
+    with pytest.raises(ValueError, match="CUDA"):
+        bdscan.train_blocks(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], 16)
