@@ -13,7 +13,7 @@
 //            [w*NPT, (w+1)*NPT) of all 32 channels (W = N / NPT warps). A
 //            warp's B and C reads are then the same address in every lane
 //            (one shared-memory wavefront), and delta is read once per lane.
-//   tiles  = T tokens (16, or 32 for 32-token blocks). x/dt/z [T x 32] and B/C
+//   tiles  = T tokens (32 for blocks of 16 or 32 tokens, else 16). x/dt/z [T x 32] and B/C
 //            [T x N] arrive in shared memory by 16-byte cp.async through a ring
 //            of stages; the CTA then computes delta = softplus(dt), delta*x and
 //            the fp32 B/C once per element.
@@ -25,8 +25,11 @@
 //            (B) the forward chain h = a h + b with its readout C.h;
 //            (C) the block-confined reverse chain g = a g + b from the kept a
 //                (and b), so the reverse costs no second exp.
-//            Recurrences and readouts use packed fp32x2 FMA (two states per
-//            instruction).
+//            For whole blocks of 4..32 tokens (N = 16) the kept a and b live in
+//            Tensor Memory (tcgen05.st / tcgen05.ld), not registers, and the
+//            forward and reverse chains run interleaved (two independent
+//            dependency chains in flight). Recurrences and readouts use packed
+//            fp32x2 FMA (two states per instruction).
 //   readout= each warp's partial sums C.(h + g) go through a padded shared-memory
 //            buffer; warp w then sums the W partials of its share of the tile's
 //            tokens, adds the skip term, applies the gate and stores y.
@@ -67,15 +70,23 @@ struct Cfg {
     static constexpr int NPT = Npt<N, MODE>::value;
     static constexpr int W = N / NPT;                 // warps per CTA (state groups)
     static constexpr int THREADS = 32 * W;
-    static constexpr int T = (MODE == kFused && (KC == 0 || KC > 16)) ? 32 : 16;   // tokens per tile
+    static constexpr int T = (MODE == kFused && (KC == 0 || KC > 16 || (KC == 16 && N == 16))) ? 32 : 16;   // tokens per tile
     static constexpr int S = T == 16 ? 4 : 3;                                    // cp.async ring depth
     static constexpr int SPAN = MODE == kFused ? (KC > 0 ? KC : T) : 16;
     static constexpr bool KEEP_B = SPAN <= 16 && N == 16;                        // keep b for phase C
     static constexpr int PER = T / W > 0 ? T / W : 1;                            // readout tokens per warp
+    // whole-block fused variants keep a block's decays and inputs in TMEM (8
+    // columns per token: a[4], b[4]). Warp w uses lane quadrant w % 4 and
+    // column range (w / 4) * WCOLS; a CTA's columns fit the SM's 512 even at
+    // the largest residency these variants reach (N = 16, K = 32: 2 CTAs x 256).
+    static constexpr int WCOLS = SPAN * 2 * NPT;
+    static constexpr int TNEED = (W / 4) * WCOLS;
+    static constexpr bool TMEM = MODE == kFused && KC > 0 && W % 4 == 0 && NPT == 4 && TNEED <= 512;
+    static constexpr int TCOLS = TNEED <= 32 ? 32 : (TNEED <= 64 ? 64 : (TNEED <= 128 ? 128 : (TNEED <= 256 ? 256 : 512)));
     // registers: the four N = 16 state-group warps of a CTA sit on the SM's four
     // sub-partitions, so 3 resident CTAs = 3 warps per sub-partition (<= 168
     // registers), enough for a 12288-channel batch in one wave on 148 SMs.
-    static constexpr int MINB = THREADS >= 512 ? 1 : (T == 16 ? 3 : 2);
+    static constexpr int MINB = THREADS >= 512 ? 1 : ((T == 16 || KC == 16) ? 3 : 2);
     static_assert(N % NPT == 0 && W <= 32, "state split");
 };
 
@@ -207,6 +218,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
     constexpr int RP = LY::RP, PER = CF::PER;
     constexpr bool KEEP_B = CF::KEEP_B;
     static_assert(T % SPAN == 0, "spans tile the tile");
+    static_assert(SPAN % 2 == 0 || !(MODE == kFused && KC > 0), "interleaved chains pair tokens");
 
     extern __shared__ __align__(16) char smem[];
     float2 *dd = reinterpret_cast<float2 *>(smem + LY::dd);
@@ -234,6 +246,17 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
         al[j] = dvalid ? __fmul_rn(a.A[d * N + n0 + j], kLog2e) : 0.f;
         h[j] = (dvalid && a.h0) ? a.h0[(b * a.D + d) * N + n0 + j] : 0.f;
         gcar[j] = 0.f;   // reverse carry across tiles (long path)
+    }
+
+    // TMEM scratch for the whole-block fused variants (warp 0 allocates)
+    __shared__ uint32_t tmem_slot;
+    uint32_t tmem_w = 0;   // this warp: lane quadrant warp % 4, columns from (warp / 4) * WCOLS
+    if constexpr (CF::TMEM) {
+        if (warp == 0) tmem_alloc(&tmem_slot, CF::TCOLS);
+        tmem_fence_before_sync();
+        __syncthreads();
+        tmem_fence_after_sync();
+        tmem_w = tmem_slot + ((uint32_t)((warp % 4) * 32) << 16) + (uint32_t)((warp / 4) * CF::WCOLS);
     }
 
     // ---- tile schedule ------------------------------------------------------
@@ -321,7 +344,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
         float yp[T];
         uint32_t endmask = 0;   // block ends inside the tile (runtime-K and forward-only)
         if (MODE == kForwardOnly || (MODE == kFused && KC == 0)) {
-            for (int64_t e = K - 1 - (t0 % K); e < tlen; e += K) endmask |= 1u << e;
+            for (int64_t e = K - 1 - (t0 % K); e < tlen; e += K) endmask |= 1u << e;   // block ends in the tile
         } else if (MODE == kLong) {
             if (!rev && (t0 + tlen) % K == 0) endmask = 1u << (tlen - 1);
         }
@@ -347,7 +370,107 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
                 }
                 yp[t] = acc;
             }
+        } else if (MODE == kFused && KC > 0) {
+            // Whole blocks (a tile holds whole blocks, since L % K == 0 and K
+            // divides T): phase A for the block, then the forward and the
+            // reverse chains interleaved -- they share only the kept decays, so
+            // two independent dependency chains are in flight. A token's y is
+            // the sum of exactly two terms, so their order does not change it.
+#pragma unroll
+            for (int sp = 0; sp < T / SPAN; ++sp) {
+                const int s0 = sp * SPAN;
+                if (s0 >= tlen) {
+#pragma unroll
+                    for (int i = 0; i < SPAN; ++i) yp[s0 + i] = 0.f;
+                    continue;
+                }
+                float gs[NPT];
+#pragma unroll
+                for (int j = 0; j < NPT; ++j) gs[j] = 0.f;
+                if constexpr (CF::TMEM) {
+                    // (A) a and b of every token of the block into this warp's TMEM lanes
+#pragma unroll
+                    for (int i = 0; i < SPAN; ++i) {
+                        float at4[NPT], bq4[NPT], v[8];
+                        decay_input<NPT>(al, ddc[(s0 + i) * kCh], Bw + (s0 + i) * N, at4, bq4);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) { v[j] = at4[j]; v[4 + j] = bq4[j]; }
+                        tmem_st8(tmem_w + i * 8, v);
+                    }
+                    tmem_wait_st();
+                    // (B)+(C), reading step i+1's operands while step i computes
+                    float cf[8], cr[8];
+                    tmem_ld8(tmem_w + 0, cf);
+                    tmem_ld8(tmem_w + (SPAN - 1) * 8, cr);
+                    tmem_wait_ld(cf, cr);
+#pragma unroll
+                    for (int i = 0; i < SPAN; ++i) {
+                        const int tf = s0 + i, ir = SPAN - 1 - i, tr = s0 + ir;
+                        float nf[8], nr[8];
+                        if (i + 1 < SPAN) {
+                            tmem_ld8(tmem_w + (i + 1) * 8, nf);
+                            tmem_ld8(tmem_w + (ir - 1) * 8, nr);
+                        }
+                        float af[NPT], bfq[NPT], ar[NPT], brq[NPT];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) { af[j] = cf[j]; bfq[j] = cf[4 + j]; ar[j] = cr[j]; brq[j] = cr[4 + j]; }
+                        const float vf = scan_step<NPT>(h, af, bfq, Cw + tf * N);
+                        const float vr = scan_step<NPT>(gs, ar, brq, Cw + tr * N);
+                        if (i < SPAN / 2) {
+                            yp[tf] = vf;
+                            yp[tr] = vr;
+                        } else {
+                            yp[tf] = __fadd_rn(yp[tf], vf);
+                            yp[tr] = __fadd_rn(yp[tr], vr);
+                        }
+                        if (i + 1 < SPAN) {
+                            tmem_wait_ld(nf, nr);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) { cf[j] = nf[j]; cr[j] = nr[j]; }
+                        }
+                    }
+                } else {
+                    constexpr int NB = KEEP_B ? SPAN : 1;
+                    float at[SPAN][NPT];
+                    float bt[NB][NPT];
+#pragma unroll
+                    for (int i = 0; i < SPAN; ++i) {   // (A)
+                        float bq[NPT];
+                        decay_input<NPT>(al, ddc[(s0 + i) * kCh], Bw + (s0 + i) * N, at[i], bq);
+                        if (KEEP_B) {
+#pragma unroll
+                            for (int j = 0; j < NPT; ++j) bt[KEEP_B ? i : 0][j] = bq[j];
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < SPAN; ++i) {   // (B) forward token i, (C) reverse token SPAN-1-i
+                        const int tf = s0 + i, ir = SPAN - 1 - i, tr = s0 + ir;
+                        float bf_[NPT], br_[NPT];
+                        if (KEEP_B) {
+#pragma unroll
+                            for (int j = 0; j < NPT; ++j) {
+                                bf_[j] = bt[KEEP_B ? i : 0][j];
+                                br_[j] = bt[KEEP_B ? ir : 0][j];
+                            }
+                        } else {
+                            input_only<NPT>(ddc[tf * kCh].y, Bw + tf * N, bf_);
+                            input_only<NPT>(ddc[tr * kCh].y, Bw + tr * N, br_);
+                        }
+                        const float vf = scan_step<NPT>(h, at[i], bf_, Cw + tf * N);
+                        const float vr = scan_step<NPT>(gs, at[ir], br_, Cw + tr * N);
+                        if (i < SPAN / 2) {
+                            yp[tf] = vf;
+                            yp[tr] = vr;
+                        } else {
+                            yp[tf] = __fadd_rn(yp[tf], vf);
+                            yp[tr] = __fadd_rn(yp[tr], vr);
+                        }
+                    }
+                }
+                write_boundary(t0 + s0 + SPAN - 1);
+            }
         } else {
+            // forward-only, and fused with a runtime block length (<= 32)
             constexpr bool REV = MODE == kFused;
             constexpr int NB = KEEP_B ? SPAN : 1;
 #pragma unroll
@@ -380,7 +503,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
                             input_only<NPT>(ddc[t * kCh].y, Bw + t * N, bq);
                         }
                         acc = scan_step<NPT>(h, at[i], bq, Cw + t * N);
-                        if (MODE == kFused && KC > 0 ? (i == SPAN - 1) : ((endmask >> t) & 1u)) write_boundary(t0 + t);
+                        if ((endmask >> t) & 1u) write_boundary(t0 + t);
                     }
                     yp[t] = acc;
                 }
@@ -392,7 +515,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
                     for (int i = SPAN - 1; i >= 0; --i) {   // (C)
                         const int t = s0 + i;
                         if (whole || t < tlen) {
-                            if (KC == 0 && ((endmask >> t) & 1u)) {
+                            if ((endmask >> t) & 1u) {
 #pragma unroll
                                 for (int j = 0; j < NPT; ++j) gs[j] = 0.f;
                             }
@@ -463,6 +586,12 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
         }
     }
     cp_async_wait<0>();
+    if constexpr (CF::TMEM) {   // every warp's TMEM loads completed (waited) inside its last block
+        tmem_fence_before_sync();
+        __syncthreads();
+        tmem_fence_after_sync();
+        if (warp == 0) tmem_dealloc(tmem_slot, CF::TCOLS);
+    }
 
     if (a.h_out && dvalid) {
         float *p = a.h_out + (b * a.D + d) * N + n0;
