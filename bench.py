@@ -334,6 +334,228 @@ def run_ours(args):
     return 0
 
 
+# ------------------------------------------------------- inference workloads
+def step_bytes(w) -> int:
+    """Algorithmic bytes of one block step: x, dt in, y out, B, C, A, Dskip, cache read."""
+    s = 2 if w.io == "bf16" else 4
+    return (w.batch * w.K * w.D * 3 * s + w.batch * w.K * w.N * 2 * s + 4 * w.D * w.N + 4 * w.D
+            + 4 * w.batch * w.D * w.N)
+
+
+def commit_bytes(w) -> int:
+    s = 2 if w.io == "bf16" else 4
+    return w.batch * w.K * w.D * 2 * s + w.batch * w.K * w.N * 2 * s + 4 * w.D * w.N + 8 * w.batch * w.D * w.N
+
+
+def prefill_bytes(w, L) -> int:
+    s = 2 if w.io == "bf16" else 4
+    return w.batch * L * w.D * 3 * s + w.batch * L * w.N * 2 * s + 4 * w.D * w.N + 4 * w.D + 4 * w.batch * w.D * w.N
+
+
+def run_inference(args, name):
+    """Block-diffusion inference at a long context: prefill (forward-only scan of
+    the context), then per block `steps` denoising steps (forward from the cache
+    plus in-block reverse) and one commit. Reports the prefill, the single step
+    (inputs from a rotating pool larger than twice L2, so they come from HBM) and
+    the whole denoise loop replayed as a CUDA graph."""
+    import torch
+    from selective_ssm_scan_mamba_b200 import bdscan
+    w = I.WORKLOADS[name]
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+    L, K = w.L, w.K
+
+    def up(a):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.to(dev)
+
+    p = I.make_params(w.seed, w.D, w.N)
+    A, Dk = up(p["A"]), up(p["Dskip"])
+    ctx = {k: torch.empty((w.batch, L, w.D if k in ("x", "dt") else w.N), dtype=torch.bfloat16, device=dev)
+           for k in ("x", "dt", "B", "C")}
+    span = 8 * I.CHUNK
+    for t0 in range(0, L, span):
+        n = min(span, L - t0)
+        sq = I.make_sequence(w.seed, w.batch, n, w.D, w.N, w.io, stream=("context",), t0=t0)
+        for k in ctx:
+            ctx[k][:, t0:t0 + n] = up(sq[k])
+    y_ctx = torch.empty((w.batch, L, w.D), dtype=torch.bfloat16, device=dev)
+    cache = torch.empty((w.batch, w.D, w.N), dtype=torch.float32, device=dev)
+
+    def prefill():
+        bdscan.prefill(ctx["x"], ctx["dt"], A, ctx["B"], ctx["C"], Dk, K, y=y_ctx, h_out=cache)
+
+    ws = torch.empty(max(16, bdscan.prefill_chunked_workspace_bytes(ctx["x"], ctx["B"], K)), dtype=torch.uint8,
+                     device=dev)
+
+    def prefill_chunked():
+        bdscan.prefill_chunked(ctx["x"], ctx["dt"], A, ctx["B"], ctx["C"], Dk, K, y=y_ctx, h_out=cache, ws=ws)
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn, reps=5):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps
+
+    prefill_seq_ms = timed(prefill)
+    prefill_ms = timed(prefill_chunked)
+
+    # rotating pool of noisy block inputs, > 2x L2
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    per = step_bytes(w)
+    pool_n = max(64, int(2.2 * l2 / per) + 1)
+    total_steps = w.blocks * w.steps
+    nz = I.make_sequence(w.seed, w.batch, K * pool_n, w.D, w.N, w.io, stream=("noisy", 0, 0))
+    pool = {k: up(v).view(w.batch, pool_n, K, -1).transpose(0, 1).contiguous() for k, v in nz.items()}
+    cl = I.make_sequence(w.seed, w.batch, K * w.blocks, w.D, w.N, w.io, stream=("context",), t0=L)
+    clean = {k: up(v).view(w.batch, w.blocks, K, -1).transpose(0, 1).contiguous() for k, v in cl.items()}
+    y_step = torch.empty((w.batch, K, w.D), dtype=torch.bfloat16, device=dev)
+
+    def step(i):
+        q = {k: v[i % pool_n] for k, v in pool.items()}
+        bdscan.block_step(q["x"], q["dt"], A, q["B"], q["C"], Dk, cache, y=y_step)
+
+    for i in range(10):
+        step(i)
+    torch.cuda.synchronize(dev)
+    n_meas = min(pool_n, 200)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_meas)]
+    for i in range(n_meas):
+        evs[i][0].record()
+        step(i)
+        evs[i][1].record()
+    torch.cuda.synchronize(dev)
+    step_us = statistics.median(a.elapsed_time(b) for a, b in evs) * 1e3
+
+    # the whole denoise loop (all blocks: steps + commit) as one CUDA graph
+    cache0 = cache.clone()
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        for i in range(2):   # warm up on the capture stream
+            step(i)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for j in range(w.blocks):
+                for st in range(w.steps):
+                    step(j * w.steps + st)
+                c = {k: v[j] for k, v in clean.items()}
+                bdscan.commit_block(c["x"], c["dt"], A, c["B"], c["C"], Dk, cache)
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize(dev)
+    loop_ms = []
+    for _ in range(3):
+        cache.copy_(cache0)
+        torch.cuda.synchronize(dev)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        loop_ms.append(e0.elapsed_time(e1))
+    loop_ms = statistics.median(loop_ms)
+    del g
+    launches = total_steps + w.blocks
+
+    # the full-sequence bidirectional comparator: one denoising step re-runs
+    # the reverse scan over the whole context + block (DiffuMamba-style mixing)
+    full_ms = None
+    if w.batch * (L + K) * w.D * 2 * 3 < 40e9:
+        fx = {k: torch.cat([ctx[k], pool[k][0]], dim=1).contiguous() for k in ctx}
+        fy = torch.empty((w.batch, L + K, w.D), dtype=torch.bfloat16, device=dev)
+
+        def full_step():
+            bdscan.full_bidirectional(fx["x"], fx["dt"], A, fx["B"], fx["C"], Dk, y=fy)
+
+        full_step()
+        torch.cuda.synchronize(dev)
+        e0.record()
+        for _ in range(3):
+            full_step()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        full_ms = e0.elapsed_time(e1) / 3
+        del fx, fy
+    line = {
+        "metric": METRIC, "workload": name, "n_gpus": 1, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": name, "batch": w.batch, "context": L, "d_inner": w.D, "d_state": w.N, "block": K,
+                   "steps_per_block": w.steps, "blocks": w.blocks, "io_dtype": w.io},
+        "prefill": {"ms": prefill_ms, "kind": "time-chunked (bdscan_prefill_chunked)",
+                    "sequential_ms": prefill_seq_ms, "workspace_bytes": int(ws.numel()),
+                    "tokens_per_s": w.batch * L / (prefill_ms * 1e-3),
+                    "hbm_gbs": prefill_bytes(w, L) / (prefill_ms * 1e-3) / 1e9,
+                    "hbm_frac": prefill_bytes(w, L) / (prefill_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                    "ex2_frac": w.batch * L * w.D * w.N / (prefill_ms * 1e-3) / 1e9 /
+                                (EX2_PER_CLK_SM * SM_COUNT * peaks["sm_max_mhz"] * 1e-3)},
+        "step": {"us": step_us, "scanned_tokens_per_s": w.batch * K / (step_us * 1e-6),
+                 "algorithmic_bytes": per, "hbm_gbs": per / (step_us * 1e-6) / 1e9,
+                 "hbm_frac": per / (step_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                 "inputs": f"rotating pool of {pool_n} step inputs ({pool_n * per / 1e6:.0f} MB > 2x L2)"},
+        "loop": {"ms": loop_ms, "graph_launches": launches, "us_per_launch": loop_ms * 1e3 / launches,
+                 "committed_tokens_per_s": w.batch * K * w.blocks / (loop_ms * 1e-3),
+                 "scanned_tokens_per_s": w.batch * K * launches / (loop_ms * 1e-3),
+                 "hbm_gbs": (total_steps * per + w.blocks * commit_bytes(w)) / (loop_ms * 1e-3) / 1e9},
+        "full_sequence_step": None if full_ms is None else {
+            "ms": full_ms, "tokens": L + K,
+            "vs_block_step": full_ms * 1e3 / step_us,
+            "note": "forward + reverse scan over context + active block per denoising step"},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_stack(args):
+    """24-layer N = 64 stack: one full-block pass per layer (per-layer A, Dskip),
+    for each block size; tokens/s = batch * L * layers / time."""
+    import torch
+    from selective_ssm_scan_mamba_b200 import bdscan
+    w = I.WORKLOADS["stack350m"]
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+
+    def up(a):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.to(dev)
+
+    s = I.make_sequence(w.seed, w.batch, w.L, w.D, w.N, w.io)
+    g = {k: up(v) for k, v in s.items()}
+    params = [I.make_params(w.seed, w.D, w.N, layer=l) for l in range(w.layers)]
+    As = [up(q["A"]) for q in params]
+    Ds = [up(q["Dskip"]) for q in params]
+    y = torch.empty((w.batch, w.L, w.D), dtype=torch.bfloat16, device=dev)
+    res = {}
+    for K in I.STACK_BLOCK_SIZES:
+        def layers():
+            for l in range(w.layers):
+                bdscan.train_blocks(g["x"], g["dt"], As[l], g["B"], g["C"], Ds[l], K, y=y)
+        layers()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        layers()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1)
+        per_layer = ms / w.layers
+        res[str(K)] = {"ms_24_layers": ms, "tokens_per_s": w.batch * w.L * w.layers / (ms * 1e-3),
+                       "ex2_frac": w.batch * w.L * w.D * w.N / (per_layer * 1e-3) / 1e9 /
+                                   (EX2_PER_CLK_SM * SM_COUNT * peaks["sm_max_mhz"] * 1e-3),
+                       "hbm_frac": algorithmic_bytes(w, boundary=False, h_out=False) / (per_layer * 1e-3) / 1e9
+                                   / peaks["hbm_gbs"]}
+    print(json.dumps({"metric": METRIC, "workload": "stack350m", "config": {"batch": w.batch, "seq_len": w.L,
+                      "d_inner": w.D, "d_state": w.N, "layers": w.layers, "io_dtype": w.io},
+                      "by_block": res}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -342,7 +564,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
+    ap.add_argument("--workload", default="train", choices=["train", "step65k", "step262k", "stack350m"],
+                    help="train: the headline line; the others print their own measurement lines")
     args = ap.parse_args()
+    if args.workload in ("step65k", "step262k"):
+        return run_inference(args, args.workload)
+    if args.workload == "stack350m":
+        return run_stack(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

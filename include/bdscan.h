@@ -37,7 +37,8 @@
  *
  * Conventions shared by every entry point:
  *   - All pointers are device pointers owned by the caller; the library
- *     allocates nothing, keeps no global device state and never synchronises.
+ *     allocates nothing and never synchronises; scratch memory, where an
+ *     entry point needs it, is passed in by the caller.
  *     Work is queued on `stream` (NULL = the legacy default stream) and the
  *     call returns without waiting for it.
  *   - Every pointer must be 16-byte aligned. D must be a multiple of 8 for
@@ -70,6 +71,7 @@ typedef enum {
     BDSCAN_ERR_UNSUPPORTED = 2,  /* N not 16/64, D not a multiple of the vector width,
                                     K > 768 for a pass with a reverse scan */
     BDSCAN_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned */
+    BDSCAN_ERR_WORKSPACE = 4,    /* workspace missing or smaller than the size the library asks for */
     BDSCAN_ERR_CUDA = 5          /* a kernel launch failed; see bdscan_last_cuda_error() */
 } bdscan_status;
 
@@ -117,6 +119,27 @@ int bdscan_prefill(const bdscan_dims *dims, const bdscan_inputs *in,
                    const float *h0, void *y, float *h_out, float *boundary,
                    bdscan_stream_t stream);
 
+/* Time-chunked prefill for contexts with too few channels to fill the GPU
+ * (fewer (batch, 32-channel) rows than SMs, e.g. one sequence of 65,536
+ * tokens x 1536 channels). Same outputs as
+ * bdscan_prefill, computed in two passes over chunks of the context: pass 1
+ * scans every chunk from a zero state and records its end state and the
+ * product of its decays; pass 2 rescans every chunk from the state composed
+ * from the chunks before it (h_c = P_{c-1} h_{c-1} + H_{c-1}), writing y, the
+ * block-boundary states and h_out. The composition reassociates the
+ * recurrence, so the states agree with the sequential scan within fp32
+ * rounding, not bit for bit (use bdscan_prefill where the cache must equal a
+ * commit chain exactly). Two exps per (token, channel, state). When a single
+ * chunk already fills the device the call runs bdscan_prefill's sequential
+ * scan instead (workspace size 0).
+ * ws: device scratch of bdscan_prefill_chunked_workspace(dims) bytes (the
+ * size depends on the current device's SM count), 16-byte aligned, owned by
+ * the caller, not preserved; BDSCAN_ERR_WORKSPACE if it is missing or too
+ * small. */
+size_t bdscan_prefill_chunked_workspace(const bdscan_dims *dims);
+int bdscan_prefill_chunked(const bdscan_dims *dims, const bdscan_inputs *in, const float *h0, void *y,
+                           float *h_out, float *boundary, void *ws, size_t ws_bytes, bdscan_stream_t stream);
+
 /* One denoising step of the active block (dims.seqlen == dims.block): forward
  * scan resumed from h_cache plus the in-block reverse scan from zero;
  * y = (y_fwd + y_rev) * gate. h_cache is only read.
@@ -132,6 +155,36 @@ int bdscan_block_step(const bdscan_dims *dims, const bdscan_inputs *in,
  * scanning the clean prefix, gist.science technical summary, "Methodik". */
 int bdscan_commit_block(const bdscan_dims *dims, const bdscan_inputs *in,
                         float *h_cache, void *y, bdscan_stream_t stream);
+
+/* Two-stream all-block training pass (clean prefix stream + noisy active
+ * blocks). The clean stream is scanned forward only, as the cached prefix
+ * operator: y_clean = y_fwd * gate (NULL = not written), boundary receives the
+ * state after every clean block (required: these are the caches), h_out the
+ * final state (NULL = not written). Every noisy block j then resumes the
+ * forward scan from the clean cache at its start (h0 for block 0; NULL = zero)
+ * and adds its block-confined reverse scan: y_noisy = (y_fwd + y_rev) * gate.
+ * Both streams share dims; A and Dskip are read from each stream's inputs
+ * (normally the same arrays); boundary must not alias h0. Two launches on
+ * `stream`, no scratch memory. With noisy == clean this is
+ * bdscan_train_blocks. Source: training protocol, gist.science technical
+ * summary, "Methodik" (the prefix cache is built by scanning the clean
+ * prefix; block losses are computed on top of it). */
+int bdscan_train_two_stream(const bdscan_dims *dims, const bdscan_inputs *clean, const bdscan_inputs *noisy,
+                            const float *h0, void *y_clean, void *y_noisy, float *boundary, float *h_out,
+                            bdscan_stream_t stream);
+
+/* Full-sequence bidirectional pass (the DiffuMamba-style mixing that the
+ * block-confined design replaces): forward scan over all L tokens from h0 plus
+ * a reverse scan over all L tokens from zero, y = (y_fwd + y_rev) * gate
+ * (required), h_out = final forward state (NULL = not written). Equal to
+ * bdscan_train_blocks with K = L, for any L. Two launches and no scratch: the
+ * forward pass writes y_fwd + Dskip x into y, the reverse pass adds y_rev +
+ * Dskip x and applies the gate in place (so bf16 y is rounded twice).
+ * dims.block must divide L (any value; only the block-free passes run).
+ * Source: the full-sequence reverse scan of earlier hybrids, abstract and
+ * gist.science technical summary, "Problemstellung". */
+int bdscan_full_bidirectional(const bdscan_dims *dims, const bdscan_inputs *in, const float *h0, void *y,
+                              float *h_out, bdscan_stream_t stream);
 
 /* Human-readable name of a bdscan_status value (static storage). */
 const char *bdscan_status_string(int status);

@@ -11,5 +11,5 @@ matrix form, invariants, planted-mistake checks).
 """
 from .oracle import (  # noqa: F401
     decode, forward, reverse_blocks, train_blocks, prefill, block_step,
-    commit_block, bruteforce, softplus, load,
+    commit_block, bruteforce, softplus, load, two_stream,
 )

@@ -129,3 +129,30 @@ def bruteforce(x, dt, A, B, C_, Dskip, K, z=None, h0=None, dt_softplus=True, mut
     if rc != 0:
         raise ValueError("oracle_bruteforce rejected its arguments")
     return {"y": y, "boundary": bnd}
+
+
+def two_stream(clean, noisy, A, Dskip, K, h0=None, z_noisy=None, dt_softplus=True, mutant=0):
+    """All-block training with separate clean and noisy streams.
+
+    clean / noisy: dicts with x, dt, B, C ([Bt, L, ...] each). The clean stream
+    is scanned forward only (the prefix operator): its outputs y_clean and the
+    state after every block, the caches. Noisy block j resumes the forward scan
+    from the clean cache at its start (h0 for j = 0) and adds its block-confined
+    reverse scan: y_noisy = (y_fwd + y_rev) * gate. Returns dict(y_clean,
+    y_noisy, boundary, h_out).
+    """
+    f = forward(clean["x"], clean["dt"], A, clean["B"], clean["C"], Dskip, K, h0=h0,
+                dt_softplus=dt_softplus, mutant=mutant)
+    Bt, L = np.asarray(noisy["x"]).shape[:2]
+    D = np.asarray(noisy["x"]).shape[2]
+    N = np.asarray(noisy["B"]).shape[2]
+    y_noisy = np.zeros((Bt, L, D))
+    for j in range(L // K):
+        sl = slice(j * K, (j + 1) * K)
+        hj = (np.zeros((Bt, D, N)) if h0 is None else decode(h0)) if j == 0 else f["boundary"][:, j - 1]
+        blk = {k: np.ascontiguousarray(np.asarray(noisy[k])[:, sl]) for k in ("x", "dt", "B", "C")}
+        zj = None if z_noisy is None else np.ascontiguousarray(np.asarray(z_noisy)[:, sl])
+        y_noisy[:, sl] = block_step(blk["x"], blk["dt"], A, blk["B"], blk["C"], Dskip, hj, z=zj,
+                                    dt_softplus=dt_softplus, mutant=mutant)
+    return {"y_clean": _combine(f["y_fwd"], None, None, mutant), "y_noisy": y_noisy,
+            "boundary": f["boundary"], "h_out": f["h_out"]}

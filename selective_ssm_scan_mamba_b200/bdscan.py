@@ -20,7 +20,7 @@ _lib = ct.CDLL(_LIB_PATH)
 
 F32, BF16 = 0, 1
 _STATUS = {0: "BDSCAN_OK", 1: "BDSCAN_ERR_INVALID_ARG", 2: "BDSCAN_ERR_UNSUPPORTED",
-           3: "BDSCAN_ERR_ALIGNMENT", 5: "BDSCAN_ERR_CUDA"}
+           3: "BDSCAN_ERR_ALIGNMENT", 4: "BDSCAN_ERR_WORKSPACE", 5: "BDSCAN_ERR_CUDA"}
 
 
 class Dims(ct.Structure):
@@ -40,8 +40,13 @@ _lib.bdscan_train_blocks.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp, _vp, _
 _lib.bdscan_prefill.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp, _vp, _vp]
 _lib.bdscan_block_step.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp]
 _lib.bdscan_commit_block.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp]
+_lib.bdscan_train_two_stream.argtypes = [_P(Dims), _P(Inputs), _P(Inputs), _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.bdscan_full_bidirectional.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp, _vp]
+_lib.bdscan_prefill_chunked.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp, _vp, _vp, ct.c_size_t, _vp]
+_lib.bdscan_prefill_chunked_workspace.argtypes = [_P(Dims)]
+_lib.bdscan_prefill_chunked_workspace.restype = ct.c_size_t
 for _f in ("bdscan_train_blocks", "bdscan_prefill", "bdscan_block_step", "bdscan_commit_block",
-           "bdscan_version"):
+           "bdscan_train_two_stream", "bdscan_full_bidirectional", "bdscan_prefill_chunked", "bdscan_version"):
     getattr(_lib, _f).restype = ct.c_int
 _lib.bdscan_status_string.argtypes = [ct.c_int]
 _lib.bdscan_status_string.restype = ct.c_char_p
@@ -161,6 +166,41 @@ def prefill(x, dt, A, B, C, Dskip, block, z=None, h0=None, dt_softplus=True,
     return y, h_out, boundary
 
 
+def prefill_chunked_workspace_bytes(x, B, block, io_dtype=None):
+    """Scratch bytes bdscan_prefill_chunked needs for these sizes on the current device."""
+    Bt, L, D = x.shape
+    dims = Dims(Bt, L, D, B.shape[-1], int(block), BF16 if x.dtype == torch.bfloat16 else F32, 1)
+    return int(_lib.bdscan_prefill_chunked_workspace(ct.byref(dims)))
+
+
+def prefill_chunked(x, dt, A, B, C, Dskip, block, z=None, h0=None, dt_softplus=True,
+                    want_y=True, y=None, h_out=None, boundary=None, want_boundary=False, ws=None):
+    """Time-chunked prefill (see include/bdscan.h): returns (y or None, h_out, boundary or None).
+
+    ws: optional uint8 device tensor of at least prefill_chunked_workspace_bytes(); allocated here if None.
+    """
+    dims, ins, (Bt, L, D, N), io, dev = _prepare(x, dt, A, B, C, Dskip, block, z, dt_softplus)
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (Bt, D, N), dev)
+    if y is None and want_y:
+        y = torch.empty((Bt, L, D), dtype=io, device=dev)
+    if y is not None:
+        _need(y, "y", io, (Bt, L, D), dev)
+    h_out = torch.empty((Bt, D, N), dtype=torch.float32, device=dev) if h_out is None else h_out
+    _need(h_out, "h_out", torch.float32, (Bt, D, N), dev)
+    if boundary is None and want_boundary:
+        boundary = torch.empty((Bt, L // int(block), D, N), dtype=torch.float32, device=dev)
+    if boundary is not None:
+        _need(boundary, "boundary", torch.float32, (Bt, L // int(block), D, N), dev)
+    need = int(_lib.bdscan_prefill_chunked_workspace(ct.byref(dims)))
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    rc = _lib.bdscan_prefill_chunked(ct.byref(dims), ct.byref(ins), _ptr(h0), _ptr(y), _ptr(h_out),
+                                     _ptr(boundary), _ptr(ws), ws.numel() * ws.element_size(), _stream(dev))
+    _check(rc, "bdscan_prefill_chunked")
+    return y, h_out, boundary
+
+
 def block_step(x, dt, A, B, C, Dskip, h_cache, z=None, dt_softplus=True, y=None):
     """One denoising step of the active block (L == block): returns y. h_cache is read only."""
     block = x.shape[1]
@@ -185,6 +225,57 @@ def commit_block(x, dt, A, B, C, Dskip, h_cache, z=None, dt_softplus=True, want_
     rc = _lib.bdscan_commit_block(ct.byref(dims), ct.byref(ins), _ptr(h_cache), _ptr(y), _stream(dev))
     _check(rc, "bdscan_commit_block")
     return y
+
+
+def train_two_stream(clean, noisy, A, Dskip, block, h0=None, dt_softplus=True, want_y_clean=True,
+                     y_clean=None, y_noisy=None, boundary=None, h_out=None, want_h_out=False):
+    """Two-stream all-block training pass.
+
+    clean, noisy: dicts with x, dt, B, C (and optionally z) tensors of one
+    shape. Returns (y_clean or None, y_noisy, boundary, h_out or None).
+    """
+    dims, cin, (Bt, L, D, N), io, dev = _prepare(clean["x"], clean["dt"], A, clean["B"], clean["C"], Dskip, block,
+                                                 clean.get("z"), dt_softplus)
+    dims2, nin, shp2, io2, dev2 = _prepare(noisy["x"], noisy["dt"], A, noisy["B"], noisy["C"], Dskip, block,
+                                           noisy.get("z"), dt_softplus)
+    if (Bt, L, D, N) != shp2 or io != io2 or dev != dev2:
+        raise ValueError("clean and noisy streams must have the same shapes, dtype and device")
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (Bt, D, N), dev)
+    if y_clean is None and want_y_clean:
+        y_clean = torch.empty((Bt, L, D), dtype=io, device=dev)
+    if y_clean is not None:
+        _need(y_clean, "y_clean", io, (Bt, L, D), dev)
+    y_noisy = torch.empty((Bt, L, D), dtype=io, device=dev) if y_noisy is None else y_noisy
+    _need(y_noisy, "y_noisy", io, (Bt, L, D), dev)
+    boundary = torch.empty((Bt, L // int(block), D, N), dtype=torch.float32, device=dev) if boundary is None else boundary
+    _need(boundary, "boundary", torch.float32, (Bt, L // int(block), D, N), dev)
+    if h_out is None and want_h_out:
+        h_out = torch.empty((Bt, D, N), dtype=torch.float32, device=dev)
+    if h_out is not None:
+        _need(h_out, "h_out", torch.float32, (Bt, D, N), dev)
+    rc = _lib.bdscan_train_two_stream(ct.byref(dims), ct.byref(cin), ct.byref(nin), _ptr(h0), _ptr(y_clean),
+                                      _ptr(y_noisy), _ptr(boundary), _ptr(h_out), _stream(dev))
+    _check(rc, "bdscan_train_two_stream")
+    return y_clean, y_noisy, boundary, h_out
+
+
+def full_bidirectional(x, dt, A, B, C, Dskip, z=None, h0=None, dt_softplus=True, y=None, h_out=None,
+                       want_h_out=False):
+    """Forward and reverse scans over the whole sequence (no blocks): returns (y, h_out or None)."""
+    L = x.shape[1]
+    dims, ins, (Bt, L, D, N), io, dev = _prepare(x, dt, A, B, C, Dskip, max(L, 1), z, dt_softplus)
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (Bt, D, N), dev)
+    y = torch.empty((Bt, L, D), dtype=io, device=dev) if y is None else y
+    _need(y, "y", io, (Bt, L, D), dev)
+    if h_out is None and want_h_out:
+        h_out = torch.empty((Bt, D, N), dtype=torch.float32, device=dev)
+    if h_out is not None:
+        _need(h_out, "h_out", torch.float32, (Bt, D, N), dev)
+    rc = _lib.bdscan_full_bidirectional(ct.byref(dims), ct.byref(ins), _ptr(h0), _ptr(y), _ptr(h_out), _stream(dev))
+    _check(rc, "bdscan_full_bidirectional")
+    return y, h_out
 
 
 def raw_library():

@@ -12,7 +12,8 @@ thread_local cudaError_t g_last_cuda = cudaSuccess;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-enum Op { kTrain, kPrefill, kStep, kCommit };
+enum Op { kTrain, kPrefill, kStep, kCommit, kCleanStream, kReverseAccumulate };
+// kCleanStream: prefill with h_out optional; kReverseAccumulate: whole-sequence reverse scan added into y
 
 int check_common(const bdscan_dims *dm, const bdscan_inputs *in) {
     if (!dm || !in) return BDSCAN_ERR_INVALID_ARG;
@@ -37,7 +38,7 @@ int check_common(const bdscan_dims *dm, const bdscan_inputs *in) {
 }
 
 template <class IO, int N, int MODE, int KC>
-int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st) {
+int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1) {
     using CF = bdk::Cfg<N, MODE, KC>;
     using LY = bdk::Layout<IO, N, MODE, KC>;
     const size_t smem = LY::base_bytes + (MODE == bdk::kLong ? (size_t)a.K * bdk::kCh * 4 : 0);
@@ -53,7 +54,7 @@ int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st) {
         if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
         done_mask.fetch_or(bit, std::memory_order_acq_rel);
     }
-    dim3 grid((unsigned)((a.D + bdk::kCh - 1) / bdk::kCh), (unsigned)batch);
+    dim3 grid((unsigned)((a.D + bdk::kCh - 1) / bdk::kCh), (unsigned)batch, gz);
     kern<<<grid, CF::THREADS, smem, st>>>(a);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
@@ -61,9 +62,10 @@ int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st) {
 }
 
 template <class IO, int N>
-int dispatch_mode(int mode, const bdk::ScanArgs &a, int64_t batch, cudaStream_t st) {
-    if (mode == bdk::kForwardOnly) return launch<IO, N, bdk::kForwardOnly, 0>(a, batch, st);
+int dispatch_mode(int mode, const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1) {
+    if (mode == bdk::kForwardOnly) return launch<IO, N, bdk::kForwardOnly, 0>(a, batch, st, gz);
     if (mode == bdk::kLong) return launch<IO, N, bdk::kLong, 0>(a, batch, st);
+    if (mode == bdk::kReverseAcc) return launch<IO, N, bdk::kReverseAcc, 0>(a, batch, st);
     switch (a.K) {
         case 4: return launch<IO, N, bdk::kFused, 4>(a, batch, st);
         case 16: return launch<IO, N, bdk::kFused, 16>(a, batch, st);
@@ -72,14 +74,20 @@ int dispatch_mode(int mode, const bdk::ScanArgs &a, int64_t batch, cudaStream_t 
     }
 }
 
+struct Chunking {   // time-chunked prefill: chunk length, chunk count, pass, workspace halves
+    int64_t len = 0, count = 1;
+    int pass = 0;
+    float *ws_h = nullptr, *ws_p = nullptr;
+};
+
 int run(Op op, const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, void *y, float *h_out,
-        float *boundary, bdscan_stream_t stream) {
+        float *boundary, bdscan_stream_t stream, const float *blk_h0 = nullptr, const Chunking *ch = nullptr) {
     int rc = check_common(dm, in);
     if (rc != BDSCAN_OK) return rc;
     if ((op == kStep || op == kCommit) && dm->seqlen != dm->block) return BDSCAN_ERR_INVALID_ARG;
     const bool any_y = dm->batch * dm->seqlen * dm->d_inner > 0;
     const bool any_state = dm->batch * dm->d_inner > 0;
-    if ((op == kTrain || op == kStep) && any_y && !y) return BDSCAN_ERR_INVALID_ARG;
+    if ((op == kTrain || op == kStep || op == kReverseAccumulate) && any_y && !y) return BDSCAN_ERR_INVALID_ARG;
     if ((op == kPrefill || op == kCommit) && any_state && !h_out) return BDSCAN_ERR_INVALID_ARG;
     if (op == kStep && any_state && !h0) return BDSCAN_ERR_INVALID_ARG;
     const void *outs[] = {h0, y, h_out, boundary};
@@ -87,7 +95,9 @@ int run(Op op, const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, 
         if (p && !aligned16(p)) return BDSCAN_ERR_ALIGNMENT;
 
     int mode;
-    if (op == kPrefill || (op == kCommit && !y)) {
+    if (op == kReverseAccumulate) {
+        mode = bdk::kReverseAcc;
+    } else if (op == kPrefill || op == kCleanStream || (op == kCommit && !y)) {
         mode = bdk::kForwardOnly;
     } else if (dm->block <= 32) {
         mode = bdk::kFused;
@@ -100,19 +110,85 @@ int run(Op op, const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, 
     bdk::ScanArgs a;
     a.x = in->x; a.dt = in->dt; a.B = in->B; a.C = in->C; a.z = in->z;
     a.A = in->A; a.Dskip = in->Dskip; a.h0 = h0;
-    a.y = y; a.h_out = h_out; a.boundary = boundary;
+    a.y = y; a.h_out = h_out; a.boundary = boundary; a.blk_h0 = blk_h0;
+    a.chunk_len = ch ? ch->len : 0;
+    a.chunk_pass = ch ? ch->pass : 0;
+    a.ws_h = ch ? ch->ws_h : nullptr;
+    a.ws_p = ch ? ch->ws_p : nullptr;
+    const unsigned gz = ch ? (unsigned)ch->count : 1u;
     a.L = dm->seqlen; a.D = dm->d_inner; a.K = (int32_t)dm->block; a.dt_softplus = dm->dt_softplus;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (dm->io_dtype == BDSCAN_BF16)
-        return dm->d_state == 16 ? dispatch_mode<__nv_bfloat16, 16>(mode, a, dm->batch, st)
-                                 : dispatch_mode<__nv_bfloat16, 64>(mode, a, dm->batch, st);
-    return dm->d_state == 16 ? dispatch_mode<float, 16>(mode, a, dm->batch, st)
-                             : dispatch_mode<float, 64>(mode, a, dm->batch, st);
+        return dm->d_state == 16 ? dispatch_mode<__nv_bfloat16, 16>(mode, a, dm->batch, st, gz)
+                                 : dispatch_mode<__nv_bfloat16, 64>(mode, a, dm->batch, st, gz);
+    return dm->d_state == 16 ? dispatch_mode<float, 16>(mode, a, dm->batch, st, gz)
+                             : dispatch_mode<float, 64>(mode, a, dm->batch, st, gz);
+}
+
+// Chunk plan of the time-chunked prefill. Chunks cost a second pass, so they
+// are used only when the (batch, 32-channel) rows alone give fewer CTAs than
+// the device has SMs; then enough chunks that the CTAs fill the device about
+// three deep, at most 64 chunks and at least 256 tokens per chunk. The chunk
+// length is a multiple of 16 tokens.
+Chunking chunk_plan(const bdscan_dims *dm) {
+    Chunking c;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t row_ctas = dm->batch * ((dm->d_inner + bdk::kCh - 1) / bdk::kCh);
+    int64_t g = (row_ctas > 0 && row_ctas < sms) ? (3 * (int64_t)sms + row_ctas - 1) / row_ctas : 1;
+    const int64_t gmax_len = dm->seqlen / 256 > 0 ? dm->seqlen / 256 : 1;
+    if (g > 64) g = 64;
+    if (g > gmax_len) g = gmax_len;
+    if (g < 1) g = 1;
+    int64_t len = (dm->seqlen + g - 1) / g;
+    len = ((len + 15) / 16) * 16;
+    if (len < 16) len = 16;
+    c.len = len;
+    c.count = (dm->seqlen + len - 1) / len;
+    if (c.count < 1) c.count = 1;
+    return c;
+}
+
+size_t chunked_ws_bytes(const bdscan_dims *dm, const Chunking &c) {
+    if (c.count <= 1) return 0;
+    return 2 * (size_t)dm->batch * (size_t)c.count * (size_t)dm->d_inner * (size_t)dm->d_state * sizeof(float);
+}
+
+// The two passes of the time-chunked prefill on caller-provided scratch
+// (ws: 2 * batch * chunks * D * N floats, 16-byte aligned).
+int prefill_chunked_on(const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, void *y, float *h_out,
+                       float *boundary, float *ws, bdscan_stream_t stream) {
+    Chunking c = chunk_plan(dm);
+    if (c.count <= 1)   // enough parallelism without chunks: the sequential scan (bit-identical caches)
+        return run(kPrefill, dm, in, h0, y, h_out, boundary, stream);
+    const size_t half = (size_t)dm->batch * c.count * dm->d_inner * dm->d_state;
+    c.ws_h = ws;
+    c.ws_p = ws + half;
+    c.pass = 1;
+    int rc = run(kCleanStream, dm, in, nullptr, nullptr, nullptr, nullptr, stream, nullptr, &c);
+    if (rc != BDSCAN_OK) return rc;
+    c.pass = 2;
+    return run(kPrefill, dm, in, h0, y, h_out, boundary, stream, nullptr, &c);
 }
 
 }  // namespace
 
 extern "C" {
+
+size_t bdscan_prefill_chunked_workspace(const bdscan_dims *dims) {
+    if (!dims || dims->batch < 0 || dims->seqlen < 0 || dims->d_inner < 0 || dims->d_state < 0) return 0;
+    return chunked_ws_bytes(dims, chunk_plan(dims));
+}
+
+int bdscan_prefill_chunked(const bdscan_dims *dims, const bdscan_inputs *in, const float *h0, void *y,
+                           float *h_out, float *boundary, void *ws, size_t ws_bytes, bdscan_stream_t stream) {
+    int rc = check_common(dims, in);
+    if (rc != BDSCAN_OK) return rc;
+    const size_t need = chunked_ws_bytes(dims, chunk_plan(dims));
+    if (need > 0 && (!ws || ws_bytes < need)) return BDSCAN_ERR_WORKSPACE;
+    if (ws && !aligned16(ws)) return BDSCAN_ERR_ALIGNMENT;
+    return prefill_chunked_on(dims, in, h0, y, h_out, boundary, static_cast<float *>(ws), stream);
+}
 
 int bdscan_train_blocks(const bdscan_dims *dims, const bdscan_inputs *in, const float *h0, void *y,
                         float *boundary, float *h_out, bdscan_stream_t stream) {
@@ -134,12 +210,42 @@ int bdscan_commit_block(const bdscan_dims *dims, const bdscan_inputs *in, float 
     return run(kCommit, dims, in, h_cache, y, h_cache, nullptr, stream);
 }
 
+int bdscan_train_two_stream(const bdscan_dims *dims, const bdscan_inputs *clean, const bdscan_inputs *noisy,
+                            const float *h0, void *y_clean, void *y_noisy, float *boundary, float *h_out,
+                            bdscan_stream_t stream) {
+    int rc = check_common(dims, noisy);
+    if (rc != BDSCAN_OK) return rc;
+    rc = check_common(dims, clean);
+    if (rc != BDSCAN_OK) return rc;
+    const bool any_block = dims->batch * dims->d_inner > 0 && dims->seqlen > 0;
+    if (any_block && !boundary) return BDSCAN_ERR_INVALID_ARG;
+    // the clean stream: forward-only scan writing the block caches (and y_clean)
+    rc = run(kCleanStream, dims, clean, h0, y_clean, h_out, boundary, stream);
+    if (rc != BDSCAN_OK) return rc;
+    // the noisy stream: every block restarts from the clean cache at its start
+    return run(kTrain, dims, noisy, h0, y_noisy, nullptr, nullptr, stream, boundary);
+}
+
+int bdscan_full_bidirectional(const bdscan_dims *dims, const bdscan_inputs *in, const float *h0, void *y,
+                              float *h_out, bdscan_stream_t stream) {
+    if (!dims || !in) return BDSCAN_ERR_INVALID_ARG;
+    bdscan_inputs ungated = *in;
+    ungated.z = nullptr;
+    // forward pass: y = y_fwd + Dskip x (ungated)
+    int rc = run(kCleanStream, dims, &ungated, h0, y, h_out, nullptr, stream);
+    if (rc != BDSCAN_OK) return rc;
+    if (dims->batch * dims->seqlen * dims->d_inner > 0 && !y) return BDSCAN_ERR_INVALID_ARG;
+    // reverse pass over the whole sequence: y = (y + y_rev + Dskip x) * gate
+    return run(kReverseAccumulate, dims, in, nullptr, y, nullptr, nullptr, stream);
+}
+
 const char *bdscan_status_string(int status) {
     switch (status) {
         case BDSCAN_OK: return "BDSCAN_OK";
         case BDSCAN_ERR_INVALID_ARG: return "BDSCAN_ERR_INVALID_ARG";
         case BDSCAN_ERR_UNSUPPORTED: return "BDSCAN_ERR_UNSUPPORTED";
         case BDSCAN_ERR_ALIGNMENT: return "BDSCAN_ERR_ALIGNMENT";
+        case BDSCAN_ERR_WORKSPACE: return "BDSCAN_ERR_WORKSPACE";
         case BDSCAN_ERR_CUDA: return "BDSCAN_ERR_CUDA";
         default: return "BDSCAN_UNKNOWN_STATUS";
     }

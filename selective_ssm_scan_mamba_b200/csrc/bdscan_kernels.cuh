@@ -10,7 +10,7 @@
 //            walks all L tokens in order; the forward state never leaves
 //            registers.
 //   warps  = lane = channel, warp = state group: warp w holds states
-//            [w*NPT, (w+1)*NPT) of all 32 channels (W = N / NPT warps). A
+//            [4w, 4w+4) of all 32 channels (W = N / 4 warps). A
 //            warp's B and C reads are then the same address in every lane
 //            (one shared-memory wavefront), and delta is read once per lane.
 //   tiles  = T tokens (32 for blocks of 16 or 32 tokens, else 16). x/dt/z [T x 32] and B/C
@@ -33,6 +33,9 @@
 //   readout= each warp's partial sums C.(h + g) go through a padded shared-memory
 //            buffer; warp w then sums the W partials of its share of the tile's
 //            tokens, adds the skip term, applies the gate and stores y.
+//   reverse= (full-sequence bidirectional comparator) the reverse scan over the
+//            whole sequence, tiles last to first, adding y_rev + Dskip x to the
+//            forward pass's y in place and applying the gate.
 //   long   = blocks longer than 32 tokens: per block, a reverse sweep over its
 //            tiles from last to first (carrying g) whose readout is staged in
 //            shared memory, then a forward sweep that adds it (two exps per
@@ -46,23 +49,35 @@ namespace bdk {
 constexpr int kCh = 32;                  // channels per CTA (one per lane)
 constexpr int kLongSmemMax = 96 * 1024;  // y_rev staging limit of the long-block path
 
-enum Mode { kForwardOnly = 0, kFused = 1, kLong = 2 };
+enum Mode { kForwardOnly = 0, kFused = 1, kLong = 2, kReverseAcc = 3 };
 
 struct ScanArgs {
     const void *x, *dt, *B, *C, *z;
     const float *A, *Dskip, *h0;
+    // optional per-block initial states (fused and long modes): block j starts
+    // its forward scan from blk_h0[b, j-1] (block 0 from h0) instead of the
+    // state carried from block j-1 -- the two-stream training pass
+    const float *blk_h0;
+    // time-chunked prefill (forward-only mode): chunk_len > 0 splits L into
+    // chunks of chunk_len tokens, one CTA row per chunk (blockIdx.z). Pass 1
+    // (chunk_pass == 1) scans each chunk from zero and writes its end state to
+    // ws_h and the product of its decays to ws_p ([batch, chunks, D, N]); pass 2
+    // (chunk_pass == 2) starts chunk c from the state folded over chunks < c.
+    int64_t chunk_len;
+    int32_t chunk_pass;
+    float *ws_h, *ws_p;
     void *y;
     float *h_out, *boundary;
     int64_t L, D;
     int32_t K, dt_softplus;
 };
 
-// States per lane: 4 where a block's decays are kept for the reverse scan;
-// the forward-only N = 16 variant spreads one state per warp (16 warps) for
-// parallelism on single-sequence prefills.
+// States per lane: 4 in every mode (one warp per 4 states). Prefills of too
+// few channels to fill the GPU get their parallelism from time chunks
+// (bdscan_prefill_chunked), not from thinner lanes.
 template <int N, int MODE>
 struct Npt {
-    static constexpr int value = (MODE == kForwardOnly && N == 16) ? 1 : 4;
+    static constexpr int value = 4;
 };
 
 template <int N, int MODE, int KC>
@@ -234,6 +249,11 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
     const int64_t d = d0 + c;
     const bool dvalid = d < a.D;
     const int64_t L = a.L, K = a.K;
+    const bool chunked = MODE == kForwardOnly && a.chunk_len > 0;
+    const int64_t nchunks = chunked ? (L + a.chunk_len - 1) / a.chunk_len : 1;
+    const int64_t cidx = chunked ? (int64_t)blockIdx.z : 0;
+    const int64_t tbeg = chunked ? cidx * a.chunk_len : 0;                           // first token of this CTA
+    const int64_t tend = chunked ? (tbeg + a.chunk_len < L ? tbeg + a.chunk_len : L) : L;
     const bool gated = a.z != nullptr;
     const bool want_y = a.y != nullptr;
     const float dskip = dvalid ? a.Dskip[d] : 0.f;
@@ -246,6 +266,24 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
         al[j] = dvalid ? __fmul_rn(a.A[d * N + n0 + j], kLog2e) : 0.f;
         h[j] = (dvalid && a.h0) ? a.h0[(b * a.D + d) * N + n0 + j] : 0.f;
         gcar[j] = 0.f;   // reverse carry across tiles (long path)
+    }
+
+    float pdec[NPT];   // running product of this chunk's decays (chunked pass 1)
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) pdec[j] = 1.f;
+    if (chunked) {
+        if (a.chunk_pass == 1) {
+#pragma unroll
+            for (int j = 0; j < NPT; ++j) h[j] = 0.f;
+        } else {
+            // h_in(c) = P(c-1) h_in(c-1) + H(c-1), from h_in(0) = h0
+            for (int64_t q = 0; q < cidx; ++q) {
+                const int64_t off = ((b * nchunks + q) * a.D + d) * N + n0;
+#pragma unroll
+                for (int j = 0; j < NPT; ++j)
+                    h[j] = dvalid ? __fmaf_rn(a.ws_p[off + j], h[j], a.ws_h[off + j]) : 0.f;
+            }
+        }
     }
 
     // TMEM scratch for the whole-block fused variants (warp 0 allocates)
@@ -264,7 +302,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
     // long: per block j, nt reverse steps (tiles nt-1 .. 0) then nt forward steps.
     const int TE = (MODE == kFused && KC == 0) ? (int)((T / K) * K) : T;
     const int64_t nt_blk = (MODE == kLong) ? (K + T - 1) / T : 1;
-    const int64_t nsteps = (MODE == kLong) ? (L / K) * 2 * nt_blk : (L + TE - 1) / TE;
+    const int64_t nsteps = (MODE == kLong) ? (L / K) * 2 * nt_blk : (tend - tbeg + TE - 1) / TE;   // kReverseAcc: TE = T
     auto tile_of = [&](int64_t s, int64_t &t0, int &tlen, bool &rev, bool &first_rev) {
         if (MODE == kLong) {
             const int64_t j = s / (2 * nt_blk), r = s % (2 * nt_blk);
@@ -274,11 +312,18 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
             t0 = j * K + i * T;
             const int64_t rem = (j + 1) * K - t0;
             tlen = (int)(rem < T ? rem : T);
+        } else if (MODE == kReverseAcc) {   // whole sequence as one block, tiles last to first
+            const int64_t nt = (L + T - 1) / T;
+            rev = true;
+            first_rev = s == 0;
+            t0 = (nt - 1 - s) * T;
+            const int64_t rem = L - t0;
+            tlen = (int)(rem < T ? rem : T);
         } else {
             rev = false;
             first_rev = false;
-            t0 = s * TE;
-            const int64_t rem = L - t0;
+            t0 = tbeg + s * TE;
+            const int64_t rem = tend - t0;
             tlen = (int)(rem < TE ? rem : TE);
         }
     };
@@ -301,6 +346,14 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
             else if constexpr (NPT == 2) *reinterpret_cast<float2 *>(p) = make_float2(h[0], h[1]);
             else p[0] = h[0];
         }
+    };
+
+    // restart the forward state at the start of block j from the per-block states
+    auto restart_h = [&](int64_t j) {
+        const float *src = j == 0 ? (a.h0 ? a.h0 + (b * a.D + d) * N + n0 : nullptr)
+                                  : a.blk_h0 + ((b * nblk + j - 1) * a.D + d) * N + n0;
+#pragma unroll
+        for (int q = 0; q < NPT; ++q) h[q] = (dvalid && src) ? src[q] : 0.f;
     };
 
     const float2 *ddc = dd + c;    // row t: ddc[t * 32]
@@ -349,7 +402,9 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
             if (!rev && (t0 + tlen) % K == 0) endmask = 1u << (tlen - 1);
         }
 
-        if (MODE == kLong && rev) {   // reverse sweep tile of a long block: decays, then the chain
+        if (MODE == kLong && !rev && a.blk_h0 && t0 % K == 0) restart_h(t0 / K);
+
+        if ((MODE == kLong || MODE == kReverseAcc) && rev) {   // reverse sweep tile: decays, then the chain
             float at[T][NPT];
 #pragma unroll
             for (int t = 0; t < T; ++t) {
@@ -384,6 +439,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
                     for (int i = 0; i < SPAN; ++i) yp[s0 + i] = 0.f;
                     continue;
                 }
+                if (a.blk_h0) restart_h((t0 + s0) / K);
                 float gs[NPT];
 #pragma unroll
                 for (int j = 0; j < NPT; ++j) gs[j] = 0.f;
@@ -469,6 +525,21 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
                 }
                 write_boundary(t0 + s0 + SPAN - 1);
             }
+        } else if (MODE == kForwardOnly && chunked && a.chunk_pass == 1) {
+            // time-chunked pass 1: the chunk's state from zero and the product of its decays
+#pragma unroll
+            for (int t = 0; t < T; ++t) {
+                if (t < tlen) {
+                    float at_[NPT], bq_[NPT];
+                    decay_input<NPT>(al, ddc[t * kCh], Bw + t * N, at_, bq_);
+#pragma unroll
+                    for (int j = 0; j < NPT; ++j) {
+                        h[j] = __fmaf_rn(at_[j], h[j], bq_[j]);
+                        pdec[j] = __fmul_rn(pdec[j], at_[j]);
+                    }
+                }
+                yp[t] = 0.f;
+            }
         } else {
             // forward-only, and fused with a runtime block length (<= 32)
             constexpr bool REV = MODE == kFused;
@@ -495,6 +566,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
                     const int t = s0 + i;
                     float acc = 0.f;
                     if (whole || t < tlen) {
+                        if (MODE == kFused && a.blk_h0 && (t0 + t) % K == 0) restart_h((t0 + t) / K);
                         float bq[NPT];
                         if (KEEP_B) {
 #pragma unroll
@@ -534,6 +606,8 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
         }
 
         // ---- readout: the W state-group partials of every (token, channel) -------
+        // (a forward-only pass without y -- commit, chunked pass 1 -- has none)
+        if (MODE == kForwardOnly && !want_y) continue;
         {
             float *rrow = red + (warp * kCh + c) * RP;   // this warp's partials for channel c
 #pragma unroll
@@ -570,7 +644,16 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
                 const int t = warp * PER + i;
                 if (t < tlen) {
                     const int yr = (int)(t0 - (t0 / K) * K) + t;   // token within its block (long path)
-                    if (MODE == kLong && rev) {
+                    if (MODE == kReverseAcc) {
+                        if (want_y && dvalid) {   // y holds y_fwd + Dskip x from the forward pass
+                            float v = __fadd_rn(to_f32(gy[(int64_t)t * a.D]), ysum[i]);
+                            v = __fmaf_rn(dskip, to_f32(xs[t * kCh + c]), v);
+                            if (gated) v = __fmul_rn(v, silu_f32(to_f32(zs[t * kCh + c])));
+                            IO o;
+                            from_f32(v, o);
+                            gy[(int64_t)t * a.D] = o;
+                        }
+                    } else if (MODE == kLong && rev) {
                         yrev[yr * kCh + c] = ysum[i];
                     } else if (want_y && dvalid) {
                         float v = ysum[i];
@@ -593,7 +676,16 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
         if (warp == 0) tmem_dealloc(tmem_slot, CF::TCOLS);
     }
 
-    if (a.h_out && dvalid) {
+    if (chunked && a.chunk_pass == 1) {
+        if (dvalid) {
+            const int64_t off = ((b * nchunks + cidx) * a.D + d) * N + n0;
+#pragma unroll
+            for (int j = 0; j < NPT; ++j) {
+                a.ws_h[off + j] = h[j];
+                a.ws_p[off + j] = pdec[j];
+            }
+        }
+    } else if (a.h_out && dvalid && cidx == nchunks - 1) {
         float *p = a.h_out + (b * a.D + d) * N + n0;
 #pragma unroll
         for (int j = 0; j < NPT; ++j) p[j] = h[j];

@@ -233,8 +233,36 @@ def check_block_locality(mutant=0):
     return True, ""
 
 
+def check_two_stream(mutant=0):
+    """Two-stream training: with noisy == clean it is the single-stream pass;
+    the clean outputs are the prefill's; a noisy block depends only on itself
+    and on the clean prefix before it."""
+    Bt, L, D, N, K = 2, 24, 3, 4, 6
+    s = _small(21, Bt, L, D, N)
+    clean = {k: s[k] for k in ("x", "dt", "B", "C")}
+    h0 = I.make_state(22, Bt, D, N)
+    r = oracle.two_stream(clean, clean, s["A"], s["Dskip"], K, h0=h0, mutant=mutant)
+    tb = oracle.train_blocks(s["x"], s["dt"], s["A"], s["B"], s["C"], s["Dskip"], K, h0=h0, mutant=mutant)
+    if not _close(r["y_noisy"], tb["y"], rtol=1e-12, atol=1e-13):
+        return False, "noisy == clean must reproduce the single-stream pass"
+    pf = oracle.prefill(s["x"], s["dt"], s["A"], s["B"], s["C"], s["Dskip"], K, h0=h0, mutant=mutant)
+    if not np.array_equal(r["y_clean"], pf["y"]) or not np.array_equal(r["boundary"], pf["boundary"]):
+        return False, "clean stream must be the forward-only prefill"
+    noisy = {k: v.copy() for k, v in I.make_sequence(23, Bt, L, D, N, "f32").items()}
+    base = oracle.two_stream(clean, noisy, s["A"], s["Dskip"], K, h0=h0, mutant=mutant)["y_noisy"]
+    j = 2
+    for k in noisy:   # change noisy block j only
+        noisy[k][:, j * K:(j + 1) * K] *= np.float32(-1.5)
+    pert = oracle.two_stream(clean, noisy, s["A"], s["Dskip"], K, h0=h0, mutant=mutant)["y_noisy"]
+    mask = np.zeros(L, bool)
+    mask[j * K:(j + 1) * K] = True
+    if not np.array_equal(pert[:, ~mask], base[:, ~mask]):
+        return False, "noisy block j must not affect other noisy blocks"
+    return True, ""
+
+
 ALL_CHECKS = [
     check_hand_example, check_softplus_closed_forms, check_block1_closed_form, check_blockL_flip,
     check_bruteforce, check_steady_state, check_linearity, check_zero_limits, check_commit_chain,
-    check_prefix_only, check_block_locality,
+    check_prefix_only, check_block_locality, check_two_stream,
 ]

@@ -206,3 +206,43 @@ def test_errors_are_raised(bd):
         bd.train_blocks(g2["x"], g2["dt"], A32, B32, B32, g2["Dskip"], 16)
     with pytest.raises(ValueError):
         bd.train_blocks(g2["x"][:, ::2], g2["dt"], g2["A"], g2["B"], g2["C"], g2["Dskip"], 16)
+
+
+@pytest.mark.parametrize("Bt,L,D,N,K,io,gated,with_h0", [
+    (1, 4096, 64, 16, 32, "bf16", False, True), (2, 3000, 40, 16, 8, "f32", True, False),
+    (1, 2048, 32, 64, 16, "bf16", True, True), (1, 520, 64, 16, 4, "f32", False, True),
+])
+def test_prefill_chunked_vs_oracle_and_sequential(bd, Bt, L, D, N, K, io, gated, with_h0):
+    s = make_case(L + D + K, Bt, L, D, N, io, gated, with_h0)
+    g = dev(s)
+    need = bd.prefill_chunked_workspace_bytes(g["x"], g["B"], K)
+    assert need > 0, "these sizes should take the chunked path"
+    y, hout, bnd = bd.prefill_chunked(g["x"], g["dt"], g["A"], g["B"], g["C"], g["Dskip"], K, z=g.get("z"),
+                                      h0=g["h0"], want_boundary=True)
+    ys, hs, bs = bd.prefill(g["x"], g["dt"], g["A"], g["B"], g["C"], g["Dskip"], K, z=g.get("z"), h0=g["h0"],
+                            want_boundary=True)
+    torch.cuda.synchronize()
+    o = oracle.prefill(s["x"], s["dt"], s["A"], s["B"], s["C"], s["Dskip"], K, z=s.get("z"), h0=s["h0"])
+    assert_c12(to_f64(y), o["y"], RTOL_Y[io], "y")
+    assert_state(to_f64(bnd), o["boundary"], "boundary states")
+    assert_state(to_f64(hout), o["h_out"], "final state")
+    assert_state(to_f64(bnd), to_f64(bs), "chunked vs sequential states")
+
+
+def test_prefill_chunked_single_chunk_is_sequential(bd):
+    s = make_case(77, 8, 256, 1536, 16, "bf16", with_h0=True)
+    g = dev(s)
+    assert bd.prefill_chunked_workspace_bytes(g["x"], g["B"], 16) == 0
+    y, h, b = bd.prefill_chunked(g["x"], g["dt"], g["A"], g["B"], g["C"], g["Dskip"], 16, h0=g["h0"], want_boundary=True)
+    ys, hs, bs = bd.prefill(g["x"], g["dt"], g["A"], g["B"], g["C"], g["Dskip"], 16, h0=g["h0"], want_boundary=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ys) and torch.equal(h, hs) and torch.equal(b, bs)
+
+
+def test_prefill_chunked_rejects_small_workspace(bd):
+    s = make_case(78, 1, 4096, 64, 16, "bf16")
+    g = dev(s)
+    need = bd.prefill_chunked_workspace_bytes(g["x"], g["B"], 16)
+    with pytest.raises(bd.BdscanError, match="WORKSPACE"):
+        bd.prefill_chunked(g["x"], g["dt"], g["A"], g["B"], g["C"], g["Dskip"], 16,
+                           ws=torch.empty(need - 16, dtype=torch.uint8, device="cuda"))
