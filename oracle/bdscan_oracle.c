@@ -53,6 +53,12 @@
  *   5 B and C swapped in the readout
  *   6 softplus replaced by exp
  *   7 forward state not carried from h0
+ * and, in the backward pass (oracle_train_blocks_backward):
+ *   8 reverse-state adjoint carried with the decay of token t, not t-1
+ *   9 forward-state adjoint restarted at every block boundary
+ *  10 decay gradient without the reverse-state term
+ *  11 dt gradient without the softplus derivative
+ *  12 initial-state gradient without the first token's decay
  */
 #include <math.h>
 #include <stdint.h>
@@ -284,6 +290,160 @@ int oracle_bruteforce(int64_t Bt, int64_t L, int64_t D, int64_t N, int64_t K,
             }
         }
     }
+    return 0;
+}
+
+/* Gradients of the all-block training output (forward over the whole
+ * sequence plus the block-confined reverse scan, combined and gated) with
+ * respect to every input, given dy = dLoss/dy [Bt, L, D]. The pages define
+ * only the forward computation; the backward pass is its adjoint, derived
+ * here by reverse-mode differentiation of the definition above:
+ *   s_t  = sum_n C_t[n] (h_t[n] + g_t[n]) + 2 Dskip x_t,  y_t = s_t * gate_t
+ *   ds_t = dy_t * gate_t,   dz_t = dy_t * s_t * silu'(z_t)
+ *   lambda_t = dL/dh_t  = ds_t C_t + a_{t+1} lambda_{t+1}   (whole sequence,
+ *              backwards from lambda_{L-1} = ds_{L-1} C_{L-1})
+ *   mu_t     = dL/dg_t  = ds_t C_t + a_{t-1} mu_{t-1}       (inside the block,
+ *              forwards from mu = ds C at the block's first token)
+ *   db_t = lambda_t + mu_t,
+ *   da_t = lambda_t h_{t-1} + mu_t g_{t+1}   (g after the block's last token = 0)
+ *   dx_t     = 2 Dskip ds_t + sum_n db_t delta_t B_t
+ *   ddelta_t = sum_n (da_t a_t A + db_t x_t B_t),  ddt_t = ddelta_t * sigmoid(dt_t)
+ *              when delta = softplus(dt), else ddelta_t
+ *   dB_t[n] = sum_d db_t delta_t x_t,  dC_t[n] = sum_d ds_t (h_t + g_t)
+ *   dA[d,n] = sum_{b,t} da_t a_t delta_t,  dDskip[d] = sum_{b,t} 2 x_t ds_t
+ *   dh0 = a_0 lambda_0.
+ * Every h_t and g_t is stored for the whole sequence (no recomputation).
+ * Outputs: dx, ddt [Bt, L, D]; dz [Bt, L, D] (only with z, else ignored);
+ * dB, dC [Bt, L, N]; dA [D, N]; dDskip [D]; dh0 [Bt, D, N] (nullable).
+ * All are overwritten. Returns 0, or -1 on bad sizes / allocation failure. */
+int oracle_train_blocks_backward(int64_t Bt, int64_t L, int64_t D, int64_t N, int64_t K,
+                                 const double *x, const double *dt, int dt_softplus,
+                                 const double *A, const double *B, const double *C,
+                                 const double *Dskip, const double *z, const double *h0,
+                                 const double *dy,
+                                 double *dx, double *ddt, double *dz, double *dB, double *dC,
+                                 double *dA, double *dDskip, double *dh0) {
+    if (Bt < 0 || L < 0 || D < 0 || N <= 0 || K <= 0 || (L % K) != 0) return -1;
+    if (!dx || !ddt || !dB || !dC || !dA || !dDskip || (z && !dz)) return -1;
+    const size_t LN = (size_t)(L > 0 ? L : 1) * (size_t)N;
+    double *dl = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    double *a = (double *)malloc(sizeof(double) * LN);    /* a_t[n] */
+    double *h = (double *)malloc(sizeof(double) * (LN + (size_t)N)); /* h_{t-1}: row t holds h_{t-1}, row L holds h_{L-1} */
+    double *g = (double *)malloc(sizeof(double) * LN);    /* g_t[n] */
+    double *ds = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    double *lam = (double *)malloc(sizeof(double) * LN);
+    double *mu = (double *)malloc(sizeof(double) * LN);
+    if (!dl || !a || !h || !g || !ds || !lam || !mu) {
+        free(dl); free(a); free(h); free(g); free(ds); free(lam); free(mu);
+        return -1;
+    }
+    memset(dB, 0, sizeof(double) * (size_t)(Bt * L * N));
+    memset(dC, 0, sizeof(double) * (size_t)(Bt * L * N));
+    memset(dA, 0, sizeof(double) * (size_t)(D * N));
+    memset(dDskip, 0, sizeof(double) * (size_t)D);
+    for (int64_t b = 0; b < Bt; ++b) {
+        for (int64_t d = 0; d < D; ++d) {
+            /* recompute the forward quantities of this channel */
+            for (int64_t t = 0; t < L; ++t) {
+                dl[t] = delta_of(dt[IDX3(b, t, d, L, D)], dt_softplus);
+                for (int64_t n = 0; n < N; ++n) a[t * N + n] = exp(dl[t] * A[d * N + n]);
+            }
+            for (int64_t n = 0; n < N; ++n) h[n] = h0 ? h0[IDX3(b, d, n, D, N)] : 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                const double xv = x[IDX3(b, t, d, L, D)];
+                for (int64_t n = 0; n < N; ++n)
+                    h[(t + 1) * N + n] = a[t * N + n] * h[t * N + n] + dl[t] * xv * B[IDX3(b, t, n, L, N)];
+            }
+            for (int64_t t = L - 1; t >= 0; --t) {
+                const int block_end = ((t + 1) % K) == 0;
+                const double xv = x[IDX3(b, t, d, L, D)];
+                for (int64_t n = 0; n < N; ++n) {
+                    const double gnext = block_end ? 0.0 : g[(t + 1) * N + n];
+                    g[t * N + n] = a[t * N + n] * gnext + dl[t] * xv * B[IDX3(b, t, n, L, N)];
+                }
+            }
+            /* output stage: s, the gate and its derivative */
+            for (int64_t t = 0; t < L; ++t) {
+                const int64_t i = IDX3(b, t, d, L, D);
+                double s = 2.0 * Dskip[d] * x[i];
+                for (int64_t n = 0; n < N; ++n)
+                    s += C[IDX3(b, t, n, L, N)] * (h[(t + 1) * N + n] + g[t * N + n]);
+                if (z) {
+                    const double sg = 1.0 / (1.0 + exp(-z[i]));
+                    ds[t] = dy[i] * z[i] * sg;
+                    dz[i] = dy[i] * s * sg * (1.0 + z[i] * (1.0 - sg));
+                } else {
+                    ds[t] = dy[i];
+                }
+            }
+            /* adjoint of the forward state, over the whole sequence */
+            for (int64_t t = L - 1; t >= 0; --t) {
+                for (int64_t n = 0; n < N; ++n) {
+                    double v = ds[t] * C[IDX3(b, t, n, L, N)];
+#if ORACLE_MUTANT == 9
+                    if (t + 1 < L && ((t + 1) % K) != 0) v += a[(t + 1) * N + n] * lam[(t + 1) * N + n];
+#else
+                    if (t + 1 < L) v += a[(t + 1) * N + n] * lam[(t + 1) * N + n];
+#endif
+                    lam[t * N + n] = v;
+                }
+            }
+            /* adjoint of the reverse state, inside each block */
+            for (int64_t t = 0; t < L; ++t) {
+                const int block_start = (t % K) == 0;
+                for (int64_t n = 0; n < N; ++n) {
+                    double v = ds[t] * C[IDX3(b, t, n, L, N)];
+#if ORACLE_MUTANT == 8
+                    if (!block_start) v += a[t * N + n] * mu[(t - 1) * N + n];
+#else
+                    if (!block_start) v += a[(t - 1) * N + n] * mu[(t - 1) * N + n];
+#endif
+                    mu[t * N + n] = v;
+                }
+            }
+            /* gradients of the inputs */
+            double dskip_acc = 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                const int64_t i = IDX3(b, t, d, L, D);
+                const double xv = x[i];
+                const int block_end = ((t + 1) % K) == 0;
+                double dxv = 2.0 * Dskip[d] * ds[t];
+                double ddl = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double Bv = B[IDX3(b, t, n, L, N)];
+                    const double dbv = lam[t * N + n] + mu[t * N + n];
+                    const double gnext = block_end ? 0.0 : g[(t + 1) * N + n];
+#if ORACLE_MUTANT == 10
+                    const double dav = lam[t * N + n] * h[t * N + n];
+                    (void)gnext;
+#else
+                    const double dav = lam[t * N + n] * h[t * N + n] + mu[t * N + n] * gnext;
+#endif
+                    dxv += dbv * dl[t] * Bv;
+                    ddl += dav * a[t * N + n] * A[d * N + n] + dbv * xv * Bv;
+                    dB[IDX3(b, t, n, L, N)] += dbv * dl[t] * xv;
+                    dC[IDX3(b, t, n, L, N)] += ds[t] * (h[(t + 1) * N + n] + g[t * N + n]);
+                    dA[d * N + n] += dav * a[t * N + n] * dl[t];
+                }
+                dx[i] = dxv;
+#if ORACLE_MUTANT == 11
+                ddt[i] = ddl;
+#else
+                ddt[i] = dt_softplus ? ddl / (1.0 + exp(-dt[i])) : ddl;
+#endif
+                dskip_acc += 2.0 * xv * ds[t];
+            }
+            dDskip[d] += dskip_acc;
+            if (dh0)
+                for (int64_t n = 0; n < N; ++n)
+#if ORACLE_MUTANT == 12
+                    dh0[IDX3(b, d, n, D, N)] = L > 0 ? lam[n] : 0.0;
+#else
+                    dh0[IDX3(b, d, n, D, N)] = L > 0 ? a[n] * lam[n] : 0.0;
+#endif
+        }
+    }
+    free(dl); free(a); free(h); free(g); free(ds); free(lam); free(mu);
     return 0;
 }
 

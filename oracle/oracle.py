@@ -28,6 +28,9 @@ def load(mutant: int = 0):
         lib.oracle_combine.restype = None
         lib.oracle_bruteforce.argtypes = [_i64] * 5 + [_dp, _dp, C.c_int, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp]
         lib.oracle_bruteforce.restype = C.c_int
+        lib.oracle_train_blocks_backward.argtypes = ([_i64] * 5 + [_dp, _dp, C.c_int] + [_dp] * 7
+                                                     + [_dp] * 8)
+        lib.oracle_train_blocks_backward.restype = C.c_int
         lib.oracle_softplus.argtypes = [C.c_double]
         lib.oracle_softplus.restype = C.c_double
         lib.oracle_mutant_id.restype = C.c_int
@@ -156,3 +159,22 @@ def two_stream(clean, noisy, A, Dskip, K, h0=None, z_noisy=None, dt_softplus=Tru
                                     dt_softplus=dt_softplus, mutant=mutant)
     return {"y_clean": _combine(f["y_fwd"], None, None, mutant), "y_noisy": y_noisy,
             "boundary": f["boundary"], "h_out": f["h_out"]}
+
+
+def train_blocks_backward(x, dt, A, B, C_, Dskip, K, dy, z=None, h0=None, dt_softplus=True, mutant=0):
+    """Gradients of train_blocks' y with respect to every input, given dy.
+
+    Returns dict(dx, ddt, dz (None without z), dB, dC, dA, dDskip, dh0), all float64.
+    """
+    x, dt, A, B, C_, Dskip, z, h0, dy = map(decode, (x, dt, A, B, C_, Dskip, z, h0, dy))
+    Bt, L, D, N = _dims(x, B)
+    out = {"dx": np.zeros((Bt, L, D)), "ddt": np.zeros((Bt, L, D)),
+           "dz": np.zeros((Bt, L, D)) if z is not None else None,
+           "dB": np.zeros((Bt, L, N)), "dC": np.zeros((Bt, L, N)), "dA": np.zeros((D, N)),
+           "dDskip": np.zeros(D), "dh0": np.zeros((Bt, D, N))}
+    rc = load(mutant).oracle_train_blocks_backward(
+        Bt, L, D, N, K, _p(x), _p(dt), int(dt_softplus), _p(A), _p(B), _p(C_), _p(Dskip), _p(z), _p(h0), _p(dy),
+        *[_p(out[k]) for k in ("dx", "ddt", "dz", "dB", "dC", "dA", "dDskip", "dh0")])
+    if rc != 0:
+        raise ValueError("oracle_train_blocks_backward rejected its arguments")
+    return out

@@ -3,7 +3,7 @@ oracle itself (a hand-derived example, closed forms, an independent matrix
 evaluation, and the invariants the method states).
 
 Each check takes the oracle build to test (``mutant`` = 0 is the real one;
-1..7 are builds with one planted mistake) and returns ``(ok, detail)``, so the
+1..12 are builds with one planted mistake) and returns ``(ok, detail)``, so the
 same checks both pin the real oracle and prove that each planted mistake is
 caught.
 """
@@ -261,8 +261,115 @@ def check_two_stream(mutant=0):
     return True, ""
 
 
+# ------------------------------------------------------------- backward pass
+_GRAD_KEYS = ("dx", "ddt", "dz", "dB", "dC", "dA", "dDskip", "dh0")
+_WRT = {"x": "dx", "dt": "ddt", "z": "dz", "B": "dB", "C": "dC", "A": "dA", "Dskip": "dDskip", "h0": "dh0"}
+
+
+def _bwd_case(seed, Bt, L, D, N, gated, with_h0, sp):
+    s = _small(seed, Bt, L, D, N, gated=gated)
+    v = {k: oracle.decode(s[k]) for k in ("x", "dt", "A", "B", "C", "Dskip")}
+    if not sp:
+        v["dt"] = np.abs(v["dt"]) * 0.3
+    v["z"] = oracle.decode(s["z"]) if gated else None
+    v["h0"] = oracle.decode(I.make_state(seed + 3, Bt, D, N)) if with_h0 else np.zeros((Bt, D, N))
+    v["dy"] = oracle.decode(I.make_state(seed + 5, Bt, L, D))
+    return v
+
+
+def _loss(v, K, sp, mutant):
+    y = oracle.train_blocks(v["x"], v["dt"], v["A"], v["B"], v["C"], v["Dskip"], K, z=v["z"], h0=v["h0"],
+                            dt_softplus=sp, mutant=mutant)["y"]
+    return float(np.sum(v["dy"] * y))
+
+
+def check_backward_finite_differences(mutant=0):
+    """Every gradient entry against a central difference of the (separately
+    pinned) forward pass, loss = sum(dy * y), on sequences that span several
+    blocks (K = 1, 2, 3, 6 over L = 6)."""
+    Bt, L, D, N = 2, 6, 2, 3
+    for K in (1, 2, 3, 6):
+        for gated, with_h0, sp in ((True, True, True), (False, False, False)):
+            v = _bwd_case(300 + K, Bt, L, D, N, gated, with_h0, sp)
+            g = oracle.train_blocks_backward(v["x"], v["dt"], v["A"], v["B"], v["C"], v["Dskip"], K, v["dy"],
+                                             z=v["z"], h0=v["h0"] if with_h0 else None, dt_softplus=sp,
+                                             mutant=mutant)
+            if not with_h0:   # gradient at the zero initial state is still defined
+                g = dict(g)
+            for name, gk in _WRT.items():
+                if v[name] is None:
+                    continue
+                arr = v[name]
+                fd = np.zeros_like(arr)
+                for i in np.ndindex(arr.shape):
+                    old = arr[i]
+                    eps = 1e-6 * max(1.0, abs(old))
+                    arr[i] = old + eps
+                    fp = _loss(v, K, sp, mutant)
+                    arr[i] = old - eps
+                    fm = _loss(v, K, sp, mutant)
+                    arr[i] = old
+                    fd[i] = (fp - fm) / (2 * eps)
+                got = g[gk]
+                scale = float(np.sqrt(np.mean(fd * fd))) + 1e-12
+                if got is None or got.shape != fd.shape or np.max(np.abs(got - fd)) > 1e-6 * scale + 1e-9:
+                    err = None if got is None or got.shape != fd.shape else float(np.max(np.abs(got - fd)) / scale)
+                    return False, f"{gk} K={K} gated={gated} h0={with_h0} sp={sp}: rel err {err}"
+    return True, ""
+
+
+def check_backward_linear_in_x(mutant=0):
+    """Ungated with h0 = 0, y is linear in x: column s of each channel's matrix
+    is y at x = unit impulse at s, from the long-double closed-form evaluation
+    (no recurrence), and dx must equal that matrix transposed times dy."""
+    Bt, L, D, N = 2, 8, 3, 4
+    for K in (1, 2, 4, 8):
+        v = _bwd_case(400 + K, Bt, L, D, N, False, False, True)
+        M = np.zeros((Bt, D, L, L))   # [b, d, t, s]
+        for s_ in range(L):
+            e = np.zeros((Bt, L, D))
+            e[:, s_, :] = 1.0
+            M[:, :, :, s_] = oracle.bruteforce(e, v["dt"], v["A"], v["B"], v["C"], v["Dskip"], K)["y"].transpose(0, 2, 1)
+        want = np.einsum("bdts,btd->bsd", M, v["dy"])
+        g = oracle.train_blocks_backward(v["x"], v["dt"], v["A"], v["B"], v["C"], v["Dskip"], K, v["dy"],
+                                         mutant=mutant)
+        if not _close(g["dx"], want, rtol=1e-11, atol=1e-12):
+            return False, f"dx K={K}: max err {np.max(np.abs(g['dx'] - want))}"
+    return True, ""
+
+
+def check_backward_homogeneity(mutant=0):
+    """Euler identities of the degree-1 homogeneities of y (loss = sum(dy * y)):
+    y is linear in (x, h0) jointly, in (C, Dskip) jointly and in (B, h0, Dskip)
+    jointly, so each set's sum of value * gradient equals the loss; and the
+    substitution A -> cA, delta -> delta/c, x -> cx, Dskip -> Dskip/c leaves y
+    unchanged (without softplus), so its derivative at c = 1 vanishes."""
+    Bt, L, D, N, K = 2, 48, 4, 8, 8
+    for gated, sp in ((True, True), (False, False)):
+        v = _bwd_case(500, Bt, L, D, N, gated, True, sp)
+        g = oracle.train_blocks_backward(v["x"], v["dt"], v["A"], v["B"], v["C"], v["Dskip"], K, v["dy"],
+                                         z=v["z"], h0=v["h0"], dt_softplus=sp, mutant=mutant)
+        loss = _loss(v, K, sp, mutant)
+        dot = lambda a, b: float(np.sum(a * b))  # noqa: E731
+        sets = {
+            "(x, h0)": dot(v["x"], g["dx"]) + dot(v["h0"], g["dh0"]),
+            "(C, Dskip)": dot(v["C"], g["dC"]) + dot(v["Dskip"], g["dDskip"]),
+            "(B, h0, Dskip)": dot(v["B"], g["dB"]) + dot(v["h0"], g["dh0"]) + dot(v["Dskip"], g["dDskip"]),
+        }
+        for name, val in sets.items():
+            if abs(val - loss) > 1e-10 * (abs(loss) + 1.0):
+                return False, f"{name}: {val} vs loss {loss}"
+        if not sp:
+            inv = dot(v["A"], g["dA"]) - dot(v["dt"], g["ddt"]) + dot(v["x"], g["dx"]) - dot(v["Dskip"], g["dDskip"])
+            scale = abs(dot(v["A"], g["dA"])) + abs(dot(v["dt"], g["ddt"])) + 1.0
+            if abs(inv) > 1e-10 * scale:
+                return False, f"A/delta rescaling invariance: {inv}"
+    return True, ""
+
+
 ALL_CHECKS = [
     check_hand_example, check_softplus_closed_forms, check_block1_closed_form, check_blockL_flip,
     check_bruteforce, check_steady_state, check_linearity, check_zero_limits, check_commit_chain,
     check_prefix_only, check_block_locality, check_two_stream,
+    check_backward_finite_differences, check_backward_linear_in_x, check_backward_homogeneity,
 ]
