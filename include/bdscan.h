@@ -140,6 +140,27 @@ size_t bdscan_prefill_chunked_workspace(const bdscan_dims *dims);
 int bdscan_prefill_chunked(const bdscan_dims *dims, const bdscan_inputs *in, const float *h0, void *y,
                            float *h_out, float *boundary, void *ws, size_t ws_bytes, bdscan_stream_t stream);
 
+/* bdscan_prefill_chunked without a workspace argument, for callers that cannot
+ * allocate device memory: code inside a framework whose memory pool owns the
+ * GPU (a raw cudaMalloc there can fail or fragment the pool), and loops that
+ * must not allocate between steps (cudaMalloc and cudaFree synchronise the
+ * device). The paper has no counterpart; this is a library convenience.
+ * Scratch is a fixed 8 MiB array in device memory that the library holds on
+ * every GPU it is loaded on until the process exits; problems whose
+ * bdscan_prefill_chunked_workspace(dims) exceeds 8 MiB return
+ * BDSCAN_ERR_WORKSPACE (use bdscan_prefill_chunked with your own buffer).
+ * The first call on a device looks up the array's device address (a CUDA
+ * runtime query, done once per device); make that first call before any
+ * stream capture. All calls share the one array and it keeps whatever the
+ * last call left there; nothing in it has to start at zero, because each
+ * call's first pass writes every entry its second pass reads. Calls that may
+ * run at the same time on the GPU (different streams with no ordering between
+ * them) race on the array and must not be issued; calls on one stream are
+ * safe. Outputs and status codes are those of
+ * bdscan_prefill_chunked; it allocates nothing. */
+int bdscan_prefill_chunked_noalloc(const bdscan_dims *dims, const bdscan_inputs *in, const float *h0, void *y,
+                                   float *h_out, float *boundary, bdscan_stream_t stream);
+
 /* One denoising step of the active block (dims.seqlen == dims.block): forward
  * scan resumed from h_cache plus the in-block reverse scan from zero;
  * y = (y_fwd + y_rev) * gate. h_cache is only read.

@@ -43,10 +43,12 @@ _lib.bdscan_commit_block.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp]
 _lib.bdscan_train_two_stream.argtypes = [_P(Dims), _P(Inputs), _P(Inputs), _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.bdscan_full_bidirectional.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp, _vp]
 _lib.bdscan_prefill_chunked.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp, _vp, _vp, ct.c_size_t, _vp]
+_lib.bdscan_prefill_chunked_noalloc.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp, _vp, _vp]
 _lib.bdscan_prefill_chunked_workspace.argtypes = [_P(Dims)]
 _lib.bdscan_prefill_chunked_workspace.restype = ct.c_size_t
 for _f in ("bdscan_train_blocks", "bdscan_prefill", "bdscan_block_step", "bdscan_commit_block",
-           "bdscan_train_two_stream", "bdscan_full_bidirectional", "bdscan_prefill_chunked", "bdscan_version"):
+           "bdscan_train_two_stream", "bdscan_full_bidirectional", "bdscan_prefill_chunked", "bdscan_prefill_chunked_noalloc",
+           "bdscan_version"):
     getattr(_lib, _f).restype = ct.c_int
 _lib.bdscan_status_string.argtypes = [ct.c_int]
 _lib.bdscan_status_string.restype = ct.c_char_p
@@ -198,6 +200,24 @@ def prefill_chunked(x, dt, A, B, C, Dskip, block, z=None, h0=None, dt_softplus=T
     rc = _lib.bdscan_prefill_chunked(ct.byref(dims), ct.byref(ins), _ptr(h0), _ptr(y), _ptr(h_out),
                                      _ptr(boundary), _ptr(ws), ws.numel() * ws.element_size(), _stream(dev))
     _check(rc, "bdscan_prefill_chunked")
+    return y, h_out, boundary
+
+
+def prefill_chunked_noalloc(x, dt, A, B, C, Dskip, block, y, h_out, z=None, h0=None, dt_softplus=True,
+                            boundary=None):
+    """Time-chunked prefill on the library's fixed 8 MiB device scratch: writes y, h_out and
+    (if given) boundary, all caller-owned, and allocates nothing. Raises BdscanError
+    (WORKSPACE) when the sizes need more scratch than that."""
+    dims, ins, (Bt, L, D, N), io, dev = _prepare(x, dt, A, B, C, Dskip, block, z, dt_softplus)
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (Bt, D, N), dev)
+    _need(y, "y", io, (Bt, L, D), dev)
+    _need(h_out, "h_out", torch.float32, (Bt, D, N), dev)
+    if boundary is not None:
+        _need(boundary, "boundary", torch.float32, (Bt, L // int(block), D, N), dev)
+    rc = _lib.bdscan_prefill_chunked_noalloc(ct.byref(dims), ct.byref(ins), _ptr(h0), _ptr(y), _ptr(h_out),
+                                             _ptr(boundary), _stream(dev))
+    _check(rc, "bdscan_prefill_chunked_noalloc")
     return y, h_out, boundary
 
 

@@ -2,6 +2,7 @@
 // Host side: argument checks, mode / template selection and launches.
 #include <atomic>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/bdscan.h"
 #include "bdscan_kernels.cuh"
@@ -171,9 +172,61 @@ int prefill_chunked_on(const bdscan_dims *dm, const bdscan_inputs *in, const flo
     return run(kPrefill, dm, in, h0, y, h_out, boundary, stream, nullptr, &c);
 }
 
+// ---- allocation-free variant of the time-chunked prefill -----------------------
+// Scratch for bdscan_prefill_chunked_noalloc: a fixed array in device global
+// memory, created when the library is loaded on a device and kept until the
+// process exits. 2^21 floats = 8 MiB per device.
+constexpr size_t kStaticScratchFloats = size_t(1) << 21;
+static __device__ __align__(256) float g_prefill_scratch[kStaticScratchFloats];
+
+// Device address of g_prefill_scratch, looked up once per device. In host code
+// the symbol name is only a handle; cudaGetSymbolAddress turns it into the
+// address the kernels must be given.
+float *static_scratch_address(int *err) {
+    static std::mutex mu;
+    static float *addr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+        *err = e != cudaSuccess ? (int)e : (int)cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_prefill_scratch);
+        if (e != cudaSuccess) {
+            *err = (int)e;
+            return nullptr;
+        }
+        addr[dev] = static_cast<float *>(p);
+    }
+    *err = 0;
+    return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
+
+int bdscan_prefill_chunked_noalloc(const bdscan_dims *dims, const bdscan_inputs *in, const float *h0, void *y,
+                                   float *h_out, float *boundary, bdscan_stream_t stream) {
+    int rc = check_common(dims, in);
+    if (rc != BDSCAN_OK) return rc;
+    const size_t need = chunked_ws_bytes(dims, chunk_plan(dims));
+    if (need > kStaticScratchFloats * sizeof(float)) return BDSCAN_ERR_WORKSPACE;   // beyond the fixed scratch
+    float *ws = nullptr;
+    if (need > 0) {
+        int err = 0;
+        ws = static_scratch_address(&err);
+        if (!ws) {
+            g_last_cuda = static_cast<cudaError_t>(err);
+            return BDSCAN_ERR_CUDA;
+        }
+    }
+    // pass 1 writes every scratch entry that pass 2 reads, so nothing needs clearing
+    return prefill_chunked_on(dims, in, h0, y, h_out, boundary, ws, stream);
+}
 
 size_t bdscan_prefill_chunked_workspace(const bdscan_dims *dims) {
     if (!dims || dims->batch < 0 || dims->seqlen < 0 || dims->d_inner < 0 || dims->d_state < 0) return 0;

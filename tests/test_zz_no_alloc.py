@@ -1,0 +1,90 @@
+"""The allocation-free time-chunked prefill (bdscan_prefill_chunked_noalloc),
+called through the C ABI, against the entry point that takes a caller
+workspace (bdscan_prefill_chunked). Two calls in a row share the library's
+fixed device scratch, so the second one also shows that nothing left there by
+the first leaks into its result."""
+import ctypes as ct
+
+import pytest
+
+from selective_ssm_scan_mamba_b200 import inputs as I
+from tests.gpu_util import RTOL_Y, assert_c12, assert_state, to_dev, to_f64
+
+SCRATCH_BYTES = 8 << 20   # the fixed scratch the header states
+
+
+def _abi():
+    from selective_ssm_scan_mamba_b200 import bdscan
+    return bdscan
+
+
+def _case(seed, Bt, L, D, N, io, gated, with_h0):
+    s = I.make_sequence(seed, Bt, L, D, N, io, gated=gated)
+    s.update(I.make_params(seed, D, N))
+    s["h0"] = I.make_state(seed + 1, Bt, D, N, scale=0.5) if with_h0 else None
+    return s
+
+
+def _dims_inputs(bd, g, Bt, L, D, N, K, io):
+    dims = bd.Dims(Bt, L, D, N, K, bd.BF16 if io == "bf16" else bd.F32, 1)
+    ins = bd.Inputs(g["x"].data_ptr(), g["dt"].data_ptr(), g["B"].data_ptr(), g["C"].data_ptr(),
+                    None if g.get("z") is None else g["z"].data_ptr(), g["A"].data_ptr(), g["Dskip"].data_ptr())
+    return dims, ins
+
+
+# (seed, Bt, L, D, N, K, io, gated, h0): both take the chunked path with under 8 MiB of scratch
+CASES = [
+    (501, 1, 8192, 512, 16, 16, "bf16", True, True),
+    (502, 2, 2048, 64, 64, 32, "f32", False, True),
+]
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
+    import torch
+    bd = _abi()
+    lib = bd.raw_library()
+    stream = torch.cuda.current_stream().cuda_stream
+    runs = []
+    for seed, Bt, L, D, N, K, io, gated, with_h0 in CASES:
+        s = _case(seed, Bt, L, D, N, io, gated, with_h0)
+        g = {k: (None if v is None else to_dev(v)) for k, v in s.items()}
+        dims, ins = _dims_inputs(bd, g, Bt, L, D, N, K, io)
+        need = int(lib.bdscan_prefill_chunked_workspace(ct.byref(dims)))
+        assert 0 < need <= SCRATCH_BYTES, need
+        ydt = torch.bfloat16 if io == "bf16" else torch.float32
+        out = dict(y=torch.empty((Bt, L, D), dtype=ydt, device="cuda"),
+                   h=torch.empty((Bt, D, N), device="cuda"),
+                   b=torch.empty((Bt, L // K, D, N), device="cuda"))
+        runs.append((s, g, dims, ins, need, out, K, io))
+    # the two allocation-free calls, back to back on one stream
+    for s, g, dims, ins, need, out, K, io in runs:
+        h0 = None if g["h0"] is None else g["h0"].data_ptr()
+        rc = lib.bdscan_prefill_chunked_noalloc(ct.byref(dims), ct.byref(ins), h0, out["y"].data_ptr(),
+                                                out["h"].data_ptr(), out["b"].data_ptr(), stream)
+        assert rc == 0, lib.bdscan_status_string(rc).decode()
+    torch.cuda.synchronize()
+    # the same problems through the entry point that takes a workspace
+    for s, g, dims, ins, need, out, K, io in runs:
+        ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+        ref = {k: torch.empty_like(v) for k, v in out.items()}
+        h0 = None if g["h0"] is None else g["h0"].data_ptr()
+        rc = lib.bdscan_prefill_chunked(ct.byref(dims), ct.byref(ins), h0, ref["y"].data_ptr(), ref["h"].data_ptr(),
+                                        ref["b"].data_ptr(), ws.data_ptr(), need, stream)
+        assert rc == 0, lib.bdscan_status_string(rc).decode()
+        torch.cuda.synchronize()
+        assert_c12(to_f64(out["y"]), to_f64(ref["y"]), RTOL_Y[io], "y")
+        assert_state(to_f64(out["h"]), to_f64(ref["h"]), "final state")
+        assert_state(to_f64(out["b"]), to_f64(ref["b"]), "boundary states")
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    # fake, never dereferenced: the size check returns before any launch
+    bd = _abi()
+    lib = bd.raw_library()
+    dims = bd.Dims(1, 8192, 4608, 64, 16, bd.BF16, 1)
+    assert int(lib.bdscan_prefill_chunked_workspace(ct.byref(dims))) > SCRATCH_BYTES
+    P = 0x100000
+    ins = bd.Inputs(P, P + 0x100, P + 0x200, P + 0x300, None, P + 0x400, P + 0x500)
+    rc = lib.bdscan_prefill_chunked_noalloc(ct.byref(dims), ct.byref(ins), None, P + 0x600, P + 0x700, None, None)
+    assert lib.bdscan_status_string(rc).decode().endswith("WORKSPACE"), rc
