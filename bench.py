@@ -17,7 +17,6 @@ bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
-import glob
 import hashlib
 import json
 import os
@@ -42,9 +41,11 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "train_traffic.json")
 
 
 def kernel_source_hash() -> str:
+    """Hash of the sources the forward scan kernel is compiled from (its
+    device code; host-side launch code and other kernels do not change it)."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "selective_ssm_scan_mamba_b200", "csrc", "*"))):
-        h.update(open(p, "rb").read())
+    for name in ("bdscan_device.cuh", "bdscan_kernels.cuh"):
+        h.update(open(os.path.join(ROOT, "selective_ssm_scan_mamba_b200", "csrc", name), "rb").read())
     return h.hexdigest()[:16]
 
 
