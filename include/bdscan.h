@@ -207,6 +207,42 @@ int bdscan_train_two_stream(const bdscan_dims *dims, const bdscan_inputs *clean,
 int bdscan_full_bidirectional(const bdscan_dims *dims, const bdscan_inputs *in, const float *h0, void *y,
                               float *h_out, bdscan_stream_t stream);
 
+/* Gradient outputs of bdscan_train_blocks_backward (all written, none accumulated). */
+typedef struct {
+    void *dx;             /* [batch, L, D] io_dtype */
+    void *ddt;            /* [batch, L, D] io_dtype, gradient w.r.t. the raw dt (through softplus if used) */
+    void *dz;             /* [batch, L, D] io_dtype; required when inputs have z, else ignored */
+    void *dB;             /* [batch, L, N] io_dtype */
+    void *dC;             /* [batch, L, N] io_dtype */
+    float *dA;            /* [D, N] fp32, summed over batch and tokens */
+    float *dDskip;        /* [D] fp32, summed over batch and tokens */
+    float *dh0;           /* [batch, D, N] fp32 gradient w.r.t. h0, or NULL */
+} bdscan_grads;
+
+/* Workspace bytes bdscan_train_blocks_backward needs for dims (0 for an
+ * unsupported d_state): per-CTA partial dB / dC rows (batch x ceil(D/32) x L
+ * x 2N fp32), per-row partial dA and dDskip, and for blocks longer than 8
+ * tokens the forward-state checkpoints at 8-token tile starts. */
+size_t bdscan_train_blocks_backward_workspace(const bdscan_dims *dims);
+
+/* Backward pass of bdscan_train_blocks: given dy = dLoss/dy, the gradients of
+ * the loss with respect to x, dt, z, B, C, A, Dskip and h0. The pages define
+ * only the forward computation (full-block objective, gist.science technical
+ * summary, "Methodik"); this is its exact adjoint:
+ *   ds_t = dy_t gate_t; lambda_t = ds_t C_t + a_{t+1} lambda_{t+1} over the
+ *   whole sequence; mu_t = ds_t C_t + a_{t-1} mu_{t-1} inside each block;
+ *   db_t = lambda_t + mu_t; da_t = lambda_t h_{t-1} + mu_t g_{t+1}.
+ * boundary = the block-boundary states bdscan_train_blocks wrote for the same
+ * inputs and h0 ([batch, L/K, D, N]; required when L > K): the forward state
+ * is recomputed from them block by block, never stored per token. Two
+ * launches on `stream` (the scan, then a fixed-order reduction of the
+ * partials: results are bitwise reproducible). ws: 16-byte aligned, at least
+ * bdscan_train_blocks_backward_workspace(dims) bytes, contents on entry
+ * ignored; dy and the gradient arrays 16-byte aligned. Any K >= 1. */
+int bdscan_train_blocks_backward(const bdscan_dims *dims, const bdscan_inputs *in, const float *h0,
+                                 const float *boundary, const void *dy, const bdscan_grads *grads, void *ws,
+                                 size_t ws_bytes, bdscan_stream_t stream);
+
 /* Human-readable name of a bdscan_status value (static storage). */
 const char *bdscan_status_string(int status);
 

@@ -34,6 +34,11 @@ class Inputs(ct.Structure):
                 ("z", ct.c_void_p), ("A", ct.c_void_p), ("Dskip", ct.c_void_p)]
 
 
+class Grads(ct.Structure):
+    _fields_ = [("dx", ct.c_void_p), ("ddt", ct.c_void_p), ("dz", ct.c_void_p), ("dB", ct.c_void_p),
+                ("dC", ct.c_void_p), ("dA", ct.c_void_p), ("dDskip", ct.c_void_p), ("dh0", ct.c_void_p)]
+
+
 _vp = ct.c_void_p
 _P = ct.POINTER
 _lib.bdscan_train_blocks.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp, _vp, _vp]
@@ -44,11 +49,15 @@ _lib.bdscan_train_two_stream.argtypes = [_P(Dims), _P(Inputs), _P(Inputs), _vp, 
 _lib.bdscan_full_bidirectional.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp, _vp]
 _lib.bdscan_prefill_chunked.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp, _vp, _vp, ct.c_size_t, _vp]
 _lib.bdscan_prefill_chunked_noalloc.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp, _vp, _vp]
+_lib.bdscan_train_blocks_backward.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp, _P(Grads), _vp, ct.c_size_t,
+                                              _vp]
+_lib.bdscan_train_blocks_backward_workspace.argtypes = [_P(Dims)]
+_lib.bdscan_train_blocks_backward_workspace.restype = ct.c_size_t
 _lib.bdscan_prefill_chunked_workspace.argtypes = [_P(Dims)]
 _lib.bdscan_prefill_chunked_workspace.restype = ct.c_size_t
 for _f in ("bdscan_train_blocks", "bdscan_prefill", "bdscan_block_step", "bdscan_commit_block",
            "bdscan_train_two_stream", "bdscan_full_bidirectional", "bdscan_prefill_chunked", "bdscan_prefill_chunked_noalloc",
-           "bdscan_version"):
+           "bdscan_train_blocks_backward", "bdscan_version"):
     getattr(_lib, _f).restype = ct.c_int
 _lib.bdscan_status_string.argtypes = [ct.c_int]
 _lib.bdscan_status_string.restype = ct.c_char_p
@@ -219,6 +228,47 @@ def prefill_chunked_noalloc(x, dt, A, B, C, Dskip, block, y, h_out, z=None, h0=N
                                              _ptr(boundary), _stream(dev))
     _check(rc, "bdscan_prefill_chunked_noalloc")
     return y, h_out, boundary
+
+
+def train_blocks_backward_workspace_bytes(x, B, block):
+    """Scratch bytes bdscan_train_blocks_backward needs for these sizes."""
+    Bt, L, D = x.shape
+    dims = Dims(Bt, L, D, B.shape[-1], int(block), BF16 if x.dtype == torch.bfloat16 else F32, 1)
+    return int(_lib.bdscan_train_blocks_backward_workspace(ct.byref(dims)))
+
+
+def train_blocks_backward(x, dt, A, B, C, Dskip, block, dy, boundary, z=None, h0=None, dt_softplus=True,
+                          want_dh0=True, grads=None, ws=None):
+    """Gradients of train_blocks' y w.r.t. every input, given dy and the forward's boundary states.
+
+    Returns dict(dx, ddt, dz (None without z), dB, dC, dA, dDskip, dh0 (None unless want_dh0)).
+    grads: optional dict of preallocated outputs; ws: optional uint8 device scratch.
+    """
+    dims, ins, (Bt, L, D, N), io, dev = _prepare(x, dt, A, B, C, Dskip, block, z, dt_softplus)
+    _need(dy, "dy", io, (Bt, L, D), dev)
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (Bt, D, N), dev)
+    if boundary is not None:
+        _need(boundary, "boundary", torch.float32, (Bt, L // int(block), D, N), dev)
+    g = dict(grads or {})
+    shapes = {"dx": ((Bt, L, D), io), "ddt": ((Bt, L, D), io), "dz": ((Bt, L, D), io), "dB": ((Bt, L, N), io),
+              "dC": ((Bt, L, N), io), "dA": ((D, N), torch.float32), "dDskip": ((D,), torch.float32),
+              "dh0": ((Bt, D, N), torch.float32)}
+    for k, (shp, dtp) in shapes.items():
+        if (k == "dz" and z is None) or (k == "dh0" and not want_dh0):
+            g[k] = None
+            continue
+        if g.get(k) is None:
+            g[k] = torch.empty(shp, dtype=dtp, device=dev)
+        _need(g[k], k, dtp, shp, dev)
+    need = int(_lib.bdscan_train_blocks_backward_workspace(ct.byref(dims)))
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    gr = Grads(*[_ptr(g[k]) for k in ("dx", "ddt", "dz", "dB", "dC", "dA", "dDskip", "dh0")])
+    rc = _lib.bdscan_train_blocks_backward(ct.byref(dims), ct.byref(ins), _ptr(h0), _ptr(boundary), _ptr(dy),
+                                           ct.byref(gr), _ptr(ws), ws.numel() * ws.element_size(), _stream(dev))
+    _check(rc, "bdscan_train_blocks_backward")
+    return g
 
 
 def block_step(x, dt, A, B, C, Dskip, h_cache, z=None, dt_softplus=True, y=None):

@@ -5,6 +5,7 @@
 #include <mutex>
 
 #include "../../include/bdscan.h"
+#include "bdscan_backward.cuh"
 #include "bdscan_kernels.cuh"
 
 namespace {
@@ -172,6 +173,61 @@ int prefill_chunked_on(const bdscan_dims *dm, const bdscan_inputs *in, const flo
     return run(kPrefill, dm, in, h0, y, h_out, boundary, stream, nullptr, &c);
 }
 
+// ---- backward pass of the all-block training scan ------------------------------
+struct BwdPlan {
+    int64_t ct, ntb, nck;
+    size_t bc, a, d, ck;   // float counts of the workspace regions (each a multiple of 4)
+};
+
+size_t round4(size_t v) { return (v + 3) & ~(size_t)3; }
+
+BwdPlan bwd_plan(const bdscan_dims *dm) {
+    BwdPlan p;
+    constexpr int TT = 8;   // tokens per tile of the backward kernel
+    p.ct = (dm->d_inner + bdk::kCh - 1) / bdk::kCh;
+    p.ntb = dm->block > TT ? (dm->block + TT - 1) / TT : 1;
+    p.nck = p.ntb > 2 ? p.ntb - 2 : 0;
+    p.bc = round4((size_t)dm->batch * p.ct * dm->seqlen * 2 * dm->d_state);
+    p.a = round4((size_t)dm->batch * dm->d_inner * dm->d_state);
+    p.d = round4((size_t)dm->batch * dm->d_inner);
+    p.ck = (size_t)dm->batch * p.ct * p.nck * (dm->d_state / 4) * bdk::kCh * 8;
+    return p;
+}
+
+size_t bwd_ws_bytes(const BwdPlan &p) { return (p.bc + p.a + p.d + p.ck) * sizeof(float); }
+
+template <class IO, int N>
+int launch_bwd(const bdk::BwdArgs &a, int64_t batch, int64_t ct, void *dB, void *dC, float *dA, float *dDskip,
+               cudaStream_t st) {
+    using CF = bdk::BwdCfg<N>;
+    using LY = bdk::BwdLayout<IO, N>;
+    auto kern = bdk::bdscan_bwd_kernel<IO, N>;
+    static std::atomic<uint64_t> done_mask{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(done_mask.load(std::memory_order_acquire) & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::bytes);
+        if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
+        done_mask.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    if (batch > 0 && ct > 0) {
+        kern<<<dim3((unsigned)ct, (unsigned)batch), CF::THREADS, LY::bytes, st>>>(a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
+    }
+    const int64_t total = batch * a.L * 2 * N + a.D * N + a.D;
+    if (total > 0) {
+        int64_t blocks = (total + 255) / 256;
+        if (blocks > 148 * 16) blocks = 148 * 16;
+        bdk::bdscan_bwd_reduce<IO, N><<<(unsigned)blocks, 256, 0, st>>>(a.ws_bc, a.ws_a, a.ws_d, dB, dC, dA, dDskip,
+                                                                        batch, a.L, a.D, ct);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
+    }
+    return BDSCAN_OK;
+}
+
 // ---- allocation-free variant of the time-chunked prefill -----------------------
 // Scratch for bdscan_prefill_chunked_noalloc: a fixed array in device global
 // memory, created when the library is loaded on a device and kept until the
@@ -241,6 +297,54 @@ int bdscan_prefill_chunked(const bdscan_dims *dims, const bdscan_inputs *in, con
     if (need > 0 && (!ws || ws_bytes < need)) return BDSCAN_ERR_WORKSPACE;
     if (ws && !aligned16(ws)) return BDSCAN_ERR_ALIGNMENT;
     return prefill_chunked_on(dims, in, h0, y, h_out, boundary, static_cast<float *>(ws), stream);
+}
+
+size_t bdscan_train_blocks_backward_workspace(const bdscan_dims *dims) {
+    if (!dims || dims->batch < 0 || dims->seqlen < 0 || dims->d_inner < 0 || dims->block < 1) return 0;
+    if (dims->d_state != 16 && dims->d_state != 64) return 0;
+    return bwd_ws_bytes(bwd_plan(dims));
+}
+
+int bdscan_train_blocks_backward(const bdscan_dims *dims, const bdscan_inputs *in, const float *h0,
+                                 const float *boundary, const void *dy, const bdscan_grads *gr, void *ws,
+                                 size_t ws_bytes, bdscan_stream_t stream) {
+    int rc = check_common(dims, in);
+    if (rc != BDSCAN_OK) return rc;
+    if (!gr) return BDSCAN_ERR_INVALID_ARG;
+    const bdscan_dims *dm = dims;
+    const bool tok = dm->batch * dm->seqlen > 0;
+    const bool elems = tok && dm->d_inner > 0;
+    if (elems && (!dy || !gr->dx || !gr->ddt)) return BDSCAN_ERR_INVALID_ARG;
+    if (elems && in->z && !gr->dz) return BDSCAN_ERR_INVALID_ARG;
+    if (tok && (!gr->dB || !gr->dC)) return BDSCAN_ERR_INVALID_ARG;
+    if (dm->d_inner > 0 && (!gr->dA || !gr->dDskip)) return BDSCAN_ERR_INVALID_ARG;
+    if (elems && dm->seqlen > dm->block && !boundary) return BDSCAN_ERR_INVALID_ARG;
+    if (dm->batch > 65535) return BDSCAN_ERR_UNSUPPORTED;
+    const void *al[] = {dy, gr->dx, gr->ddt, gr->dz, gr->dB, gr->dC};
+    for (const void *p : al)
+        if (p && !aligned16(p)) return BDSCAN_ERR_ALIGNMENT;
+    const BwdPlan p = bwd_plan(dm);
+    const size_t need = bwd_ws_bytes(p);
+    if (need > 0 && (!ws || ws_bytes < need)) return BDSCAN_ERR_WORKSPACE;
+    if (ws && !aligned16(ws)) return BDSCAN_ERR_ALIGNMENT;
+    if (dm->d_inner == 0) return BDSCAN_OK;
+    bdk::BwdArgs a{};
+    a.x = in->x; a.dt = in->dt; a.B = in->B; a.C = in->C; a.z = in->z; a.dy = dy;
+    a.A = in->A; a.Dskip = in->Dskip; a.h0 = h0; a.boundary = boundary;
+    a.dx = gr->dx; a.ddt = gr->ddt; a.dz = gr->dz; a.dh0 = gr->dh0;
+    float *w = static_cast<float *>(ws);
+    a.ws_bc = w;
+    a.ws_a = w + p.bc;
+    a.ws_d = a.ws_a + p.a;
+    a.ws_ck = p.ck ? a.ws_d + p.d : nullptr;
+    a.L = dm->seqlen; a.D = dm->d_inner; a.nck = p.nck;
+    a.K = (int32_t)dm->block; a.dt_softplus = dm->dt_softplus;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dm->io_dtype == BDSCAN_BF16)
+        return dm->d_state == 16 ? launch_bwd<__nv_bfloat16, 16>(a, dm->batch, p.ct, gr->dB, gr->dC, gr->dA, gr->dDskip, st)
+                                 : launch_bwd<__nv_bfloat16, 64>(a, dm->batch, p.ct, gr->dB, gr->dC, gr->dA, gr->dDskip, st);
+    return dm->d_state == 16 ? launch_bwd<float, 16>(a, dm->batch, p.ct, gr->dB, gr->dC, gr->dA, gr->dDskip, st)
+                             : launch_bwd<float, 64>(a, dm->batch, p.ct, gr->dB, gr->dC, gr->dA, gr->dDskip, st);
 }
 
 int bdscan_train_blocks(const bdscan_dims *dims, const bdscan_inputs *in, const float *h0, void *y,

@@ -9,6 +9,9 @@ import oracle
 # y tolerance per io dtype and the state tolerance (fp32 state in both cases)
 RTOL_Y = {"f32": 1e-5, "bf16": 2e-2}
 RTOL_STATE = 1e-6
+# gradients: per-element rule for the activation gradients (io dtype), and
+# the parameter / state gradients (fp32 sums over all tokens)
+RTOL_GRAD = {"f32": 1e-5, "bf16": 2e-2, "param": 1e-5}
 
 
 def to_dev(a, device="cuda"):
