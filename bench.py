@@ -557,6 +557,86 @@ def run_stack(args):
     return 0
 
 
+def backward_bytes(w) -> int:
+    """Algorithmic bytes of one backward call: x, dt, dy in; dx, d(dt) out;
+    B, C in and dB, dC out; the block-boundary states in; A, Dskip in and
+    dA, dDskip out (workspace partials are not counted)."""
+    s = 2 if w.io == "bf16" else 4
+    n = w.batch * w.L * w.D * s * 5
+    n += w.batch * w.L * w.N * s * 4
+    n += w.batch * (w.L // w.K) * w.D * w.N * 4
+    n += 2 * (w.D * w.N * 4 + w.D * 4)
+    return n
+
+
+def run_train_step(args):
+    """Training step of the headline workload: the all-block forward pass
+    (y + block-boundary states) and its backward pass given dy."""
+    import torch
+    from selective_ssm_scan_mamba_b200 import bdscan
+    w = I.WORKLOADS["train"]
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+
+    def up(a):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.to(dev)
+
+    s = I.make_sequence(w.seed, w.batch, w.L, w.D, w.N, w.io)
+    p = I.make_params(w.seed, w.D, w.N)
+    g = {k: up(v) for k, v in s.items()}
+    A, Dk = up(p["A"]), up(p["Dskip"])
+    dy = up(I.f32_to_bf16_bits(I.make_state(w.seed + 9, w.batch, w.L, w.D)))
+    y = torch.empty((w.batch, w.L, w.D), dtype=torch.bfloat16, device=dev)
+    bnd = torch.empty((w.batch, w.L // w.K, w.D, w.N), dtype=torch.float32, device=dev)
+    ws = torch.empty(bdscan.train_blocks_backward_workspace_bytes(g["x"], g["B"], w.K), dtype=torch.uint8,
+                     device=dev)
+    grads = {"dx": torch.empty_like(g["x"]), "ddt": torch.empty_like(g["x"]), "dB": torch.empty_like(g["B"]),
+             "dC": torch.empty_like(g["C"]), "dA": torch.empty_like(A), "dDskip": torch.empty_like(Dk),
+             "dh0": torch.empty((w.batch, w.D, w.N), dtype=torch.float32, device=dev)}
+
+    def fwd():
+        bdscan.train_blocks(g["x"], g["dt"], A, g["B"], g["C"], Dk, w.K, y=y, boundary=bnd)
+
+    def bwd():
+        bdscan.train_blocks_backward(g["x"], g["dt"], A, g["B"], g["C"], Dk, w.K, dy, bnd, grads=grads, ws=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        fwd()
+        bwd()
+    torch.cuda.synchronize(dev)
+    n = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    with ClockSampler(0) as clk:
+        for i in range(n):
+            evs[i][0].record()
+            fwd()
+            evs[i][1].record()
+            bwd()
+            evs[i][2].record()
+        torch.cuda.synchronize(dev)
+    f_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    b_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    tok = w.batch * w.L
+    ex2_peak = EX2_PER_CLK_SM * SM_COUNT * peaks["sm_max_mhz"] * 1e-3
+    elem = w.batch * w.L * w.D * w.N
+    line = {"metric": METRIC, "workload": "train_fwd_bwd", "n_gpus": 1, "steps": n, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"batch": w.batch, "seq_len": w.L, "d_inner": w.D, "d_state": w.N, "block": w.K,
+                       "io_dtype": w.io, "gated": False},
+            "forward_ms": f_ms, "backward_ms": b_ms, "step_ms": f_ms + b_ms,
+            "tokens_per_s": tok / ((f_ms + b_ms) * 1e-3),
+            "backward": {"kernels": 2, "ex2_frac": elem / (b_ms * 1e-3) / 1e9 / ex2_peak,
+                         "hbm_gbs": backward_bytes(w) / (b_ms * 1e-3) / 1e9,
+                         "hbm_frac": backward_bytes(w) / (b_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "algorithmic_bytes": backward_bytes(w),
+                         "workspace_bytes": ws.numel()},
+            "gpu_launches": 3 * n, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -565,13 +645,16 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
-    ap.add_argument("--workload", default="train", choices=["train", "step65k", "step262k", "stack350m"],
+    ap.add_argument("--workload", default="train",
+                    choices=["train", "train_fwd_bwd", "step65k", "step262k", "stack350m"],
                     help="train: the headline line; the others print their own measurement lines")
     args = ap.parse_args()
     if args.workload in ("step65k", "step262k"):
         return run_inference(args, args.workload)
     if args.workload == "stack350m":
         return run_stack(args)
+    if args.workload == "train_fwd_bwd":
+        return run_train_step(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

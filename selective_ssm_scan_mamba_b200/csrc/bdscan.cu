@@ -183,7 +183,7 @@ size_t round4(size_t v) { return (v + 3) & ~(size_t)3; }
 
 BwdPlan bwd_plan(const bdscan_dims *dm) {
     BwdPlan p;
-    constexpr int TT = 8;   // tokens per tile of the backward kernel
+    const int TT = dm->d_state == 16 ? bdk::BwdCfg<16>::TT : bdk::BwdCfg<64>::TT;   // tokens per tile
     p.ct = (dm->d_inner + bdk::kCh - 1) / bdk::kCh;
     p.ntb = dm->block > TT ? (dm->block + TT - 1) / TT : 1;
     p.nck = p.ntb > 2 ? p.ntb - 2 : 0;

@@ -31,11 +31,14 @@
 //            * over states (dx, d delta, the pre-gate sum s for dz): per-warp
 //              partials through a padded shared-memory buffer, as the forward
 //              readout does;
-//            * over channels (dB, dC, which B and C share across D): a
-//              butterfly reduce-scatter across the warp's lanes, then one
-//              partial row per CTA in the workspace, summed over the CTAs by
-//              bdscan_bwd_reduce in a fixed order (no float atomics, so the
-//              result is bitwise deterministic).
+//            * over channels (dB, dC, which B and C share across D): each
+//              lane's per-state terms go to a padded shared-memory tile that
+//              is summed over the CTA's 32 channels into one partial row per
+//              token in the workspace; bdscan_bwd_reduce sums the CTAs' rows
+//              in a fixed order (no float atomics, so the result is bitwise
+//              deterministic).
+//   block starts / ends inside a tile are bit masks formed once per tile;
+//   every per-token update runs on packed fp32x2 (two states per instruction).
 //   dA, dDskip = per-(batch row, channel) partials in the workspace, summed
 //            over the batch by bdscan_bwd_reduce.
 #pragma once
@@ -64,7 +67,7 @@ struct BwdCfg {
     static constexpr int THREADS = 32 * W;
     static constexpr int TT = 8;                       // tokens per tile
     static constexpr int S = 3;                        // cp.async ring depth
-    static constexpr int RP = TT + 4;                  // padded row of the readout buffer
+    static constexpr int BR = 2 * N + 4;               // padded per-lane row of the dB | dC tile
     static constexpr int WCOLS = TT * 16;              // TMEM columns per warp: a, b, h_prev, mu per token
     static constexpr int TNEED = ((W + 3) / 4) * WCOLS;
     static constexpr int TCOLS = TNEED <= 32 ? 32 : (TNEED <= 64 ? 64 : (TNEED <= 128 ? 128 : (TNEED <= 256 ? 256 : 512)));
@@ -76,18 +79,18 @@ struct BwdCfg {
 template <class IO, int N>
 struct BwdLayout {
     using CF = BwdCfg<N>;
-    static constexpr int TT = CF::TT, W = CF::W, RP = CF::RP;
+    static constexpr int TT = CF::TT, W = CF::W;
     static constexpr int xb = TT * kCh * (int)sizeof(IO);   // one x / dt / z / dy tile
     static constexpr int bb = TT * N * (int)sizeof(IO);     // one B / C tile
     static constexpr int stage = 4 * xb + 2 * bb;
     static constexpr int dq = CF::S * stage;                // float4 (delta, delta*x, ds, 0)  [TT][32]
     static constexpr int bf = dq + TT * kCh * 16;           // float B  [TT][N]
     static constexpr int cf = bf + TT * N * 4;              // float C  [TT][N]
-    static constexpr int red = cf + TT * N * 4;             // float [3][W][32][RP]: P, Q, S partials
-    static constexpr int bc = red + 3 * W * kCh * RP * 4;   // float [TT][2N]: the tile's dB | dC over 32 channels
-    static constexpr int dsk = bc + TT * 2 * N * 4;         // float [W][32]: dDskip partials
+    static constexpr int red = cf + TT * N * 4;             // float [3][W][TT][32]: P, Q, S partials
+    static constexpr int bc = red + 3 * W * TT * kCh * 4;   // float [TT][32][BR]: per-lane dB | dC terms
+    static constexpr int dsk = bc + TT * kCh * CF::BR * 4;  // float [W][32]: dDskip partials
     static constexpr int bytes = dsk + W * kCh * 4;
-    static_assert(xb % 16 == 0 && bb % 16 == 0 && (RP * 4) % 16 == 0, "16-byte rows");
+    static_assert(xb % 16 == 0 && bb % 16 == 0 && (CF::BR * 4) % 16 == 0, "16-byte rows");
 };
 
 // Copy tokens [t0, t0 + tlen) of x, dt, z, dy, B, C into a ring stage
@@ -131,44 +134,43 @@ __device__ __forceinline__ float sigmoid_f32(float v) {
     return rcp_approx(__fadd_rn(1.f, ex2_approx(__fmul_rn(-v, kLog2e))));
 }
 
-// Sum v[0..7] over the warp's 32 lanes, scattered: afterwards lane l holds
-// the total of v[l >> 2] (each value in four lanes). Fixed order, so the
-// result does not depend on timing.
-__device__ __forceinline__ float lane_reduce_scatter8(const float (&v)[8], int lane) {
-    float w4[4], w2[2];
-    const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float send = h16 ? v[k] : v[4 + k];
-        const float keep = h16 ? v[4 + k] : v[k];
-        w4[k] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 16));
-    }
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const float send = h8 ? w4[k] : w4[2 + k];
-        const float keep = h8 ? w4[2 + k] : w4[k];
-        w2[k] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 8));
-    }
-    const float send = h4 ? w2[0] : w2[1];
-    const float keep = h4 ? w2[1] : w2[0];
-    float r = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 4));
-    r = __fadd_rn(r, __shfl_xor_sync(0xffffffffu, r, 2));
-    r = __fadd_rn(r, __shfl_xor_sync(0xffffffffu, r, 1));
-    return r;
+__device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
+
+// Schedule of one CTA: segments from last to first; a segment of a long block
+// (K > TT) is (ntb - 1) forward tiles (phase 1) then its ntb tiles from last
+// to first (phase 2); a short-block segment is one tile of whole blocks.
+struct BwdTile {
+    int64_t t0, ts;   // first token of the tile, of its segment
+    int tlen, i, tmod;   // tokens, tile index in the segment, offset of t0 inside its block
+    bool ph1;
+};
+
+__device__ __forceinline__ BwdTile bwd_tile(int q, int r, int ntb, int64_t SL, int64_t L, bool longb, int TT) {
+    BwdTile t;
+    t.ph1 = r < ntb - 1;
+    t.i = t.ph1 ? r : 2 * ntb - 2 - r;
+    t.ts = (int64_t)q * SL;
+    t.t0 = t.ts + (int64_t)t.i * TT;
+    const int64_t send = t.ts + SL < L ? t.ts + SL : L;
+    const int64_t rem = send - t.t0;
+    t.tlen = (int)(rem < TT ? rem : TT);
+    t.tmod = longb ? t.i * TT : 0;
+    return t;
 }
 
 template <class IO, int N>
 __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bwd_kernel(const BwdArgs a) {
     using CF = BwdCfg<N>;
     using LY = BwdLayout<IO, N>;
-    constexpr int NPT = CF::NPT, W = CF::W, NT = CF::THREADS, TT = CF::TT, S = CF::S, RP = CF::RP, PER = CF::PER;
+    constexpr int NPT = CF::NPT, W = CF::W, NT = CF::THREADS, TT = CF::TT, S = CF::S, BR = CF::BR, PER = CF::PER;
+    static_assert(NPT == 4, "two packed pairs per lane");
 
     extern __shared__ __align__(16) char smem[];
     float4 *dq = reinterpret_cast<float4 *>(smem + LY::dq);
     float *Bf = reinterpret_cast<float *>(smem + LY::bf);
     float *Cf = reinterpret_cast<float *>(smem + LY::cf);
     float *red = reinterpret_cast<float *>(smem + LY::red);
-    float *bcs = reinterpret_cast<float *>(smem + LY::bc);
+    float *bcr = reinterpret_cast<float *>(smem + LY::bc);
     float *dsk = reinterpret_cast<float *>(smem + LY::dsk);
 
     const int tid = threadIdx.x, c = tid & 31, warp = tid >> 5;
@@ -176,21 +178,24 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
     const int64_t b = blockIdx.y, ct = blockIdx.x, CT = gridDim.x;
     const int64_t d0 = ct * kCh, d = d0 + c;
     const bool dvalid = d < a.D;
-    const int64_t L = a.L, K = a.K;
+    const int64_t L = a.L;
+    const int K = a.K;
     const bool gated = a.z != nullptr;
     const float dskip = dvalid ? a.Dskip[d] : 0.f;
     const float dfac = __fmul_rn(2.f, dskip);
 
-    float Av[NPT], al[NPT], rho[NPT], g[NPT], dAacc[NPT], h[NPT], nu[NPT];
+    float al[NPT];
+    float2 Av2[2], rho2[2], g2[2], dA2[2], h2[2], nu2[2];
 #pragma unroll
-    for (int j = 0; j < NPT; ++j) {
-        Av[j] = dvalid ? a.A[d * N + n0 + j] : 0.f;
-        al[j] = __fmul_rn(Av[j], kLog2e);
-        rho[j] = 0.f;   // a_{t+1} lambda_{t+1}: the forward-state adjoint carried to token t
-        g[j] = 0.f;     // g_{t+1}
-        dAacc[j] = 0.f;
-        h[j] = 0.f;
-        nu[j] = 0.f;    // a_{t-1} mu_{t-1}: the reverse-state adjoint carried to token t
+    for (int p = 0; p < 2; ++p) {
+        Av2[p] = dvalid ? make_float2(a.A[d * N + n0 + 2 * p], a.A[d * N + n0 + 2 * p + 1]) : f2(0.f);
+        al[2 * p] = __fmul_rn(Av2[p].x, kLog2e);
+        al[2 * p + 1] = __fmul_rn(Av2[p].y, kLog2e);
+        rho2[p] = f2(0.f);   // a_{t+1} lambda_{t+1}: the forward-state adjoint carried to token t
+        g2[p] = f2(0.f);     // g_{t+1}
+        dA2[p] = f2(0.f);
+        h2[p] = f2(0.f);
+        nu2[p] = f2(0.f);    // a_{t-1} mu_{t-1}: the reverse-state adjoint carried to token t
     }
     float dskacc = 0.f;
 
@@ -201,44 +206,45 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
     tmem_fence_after_sync();
     const uint32_t tw = tmem_slot + ((uint32_t)((warp % 4) * 32) << 16) + (uint32_t)((warp / 4) * CF::WCOLS);
 
-    // ---- schedule: segments from last to first; a long block's segment is
-    // (ntb - 1) forward tiles (phase 1) then ntb tiles last to first (phase 2)
     const bool longb = K > TT;
-    const int64_t SL = longb ? K : (TT / K) * K;          // segment length, a multiple of K
-    const int64_t nseg = (L + SL - 1) / SL;
-    const int64_t ntb = longb ? (K + TT - 1) / TT : 1;    // tiles per segment
-    const int64_t spseg = 2 * ntb - 1;
-    const int64_t nsteps = nseg * spseg;
-    auto tile_of = [&](int64_t s, int64_t &t0, int &tlen, bool &ph1, int64_t &i, int64_t &ts) {
-        const int64_t q = nseg - 1 - s / spseg, r = s % spseg;
-        ph1 = r < ntb - 1;
-        i = ph1 ? r : 2 * ntb - 2 - r;
-        ts = q * SL;
-        t0 = ts + i * TT;
-        const int64_t send = (q + 1) * SL < L ? (q + 1) * SL : L;
-        const int64_t rem = send - t0;
-        tlen = (int)(rem < TT ? rem : TT);
+    const int64_t SL = longb ? (int64_t)K : (int64_t)(TT / K) * K;   // segment length, a multiple of K
+    const int nseg = (int)((L + SL - 1) / SL);
+    const int ntb = longb ? (K + TT - 1) / TT : 1;                    // tiles per segment
+    const int spseg = 2 * ntb - 1;
+    const int64_t nblk = L / K;
+    // current step (q, r) and the prefetch pointer (iq, ir), S - 1 steps ahead
+    int q = nseg - 1, r = 0, iq = nseg - 1, ir = 0;
+    auto advance = [&](int &qq, int &rr) {
+        if (++rr == spseg) { rr = 0; --qq; }
     };
-    auto issue = [&](int64_t s) {
-        if (s < nsteps) {
-            int64_t t0, i, ts; int tlen; bool ph1;
-            tile_of(s, t0, tlen, ph1, i, ts);
-            stage_bwd_tile<IO, N, TT, NT>(smem + (s % S) * LY::stage, a, b, d0, t0, tlen, gated);
+    auto issue = [&](int slot) {
+        if (iq >= 0) {
+            const BwdTile tl = bwd_tile(iq, ir, ntb, SL, L, longb, TT);
+            stage_bwd_tile<IO, N, TT, NT>(smem + slot * LY::stage, a, b, d0, tl.t0, tl.tlen, gated);
+            advance(iq, ir);
         }
         cp_async_commit();
     };
-    const int64_t nblk = L / K;
-    auto init_segment = [&](int64_t ts) {   // forward state at a block start, reverse adjoint zero
-        const float *src = ts == 0 ? (a.h0 ? a.h0 + (b * a.D + d) * N + n0 : nullptr)
-                                   : a.boundary + ((b * nblk + ts / K - 1) * a.D + d) * N + n0;
-#pragma unroll
-        for (int j = 0; j < NPT; ++j) {
-            h[j] = (dvalid && src) ? src[j] : 0.f;
-            nu[j] = 0.f;
-        }
-    };
     float *ck_base = a.ws_ck ? a.ws_ck + (((b * CT + ct) * a.nck * W + warp) * kCh + c) * 8 : nullptr;
     const int64_t ck_stride = (int64_t)W * kCh * 8;   // between consecutive checkpoints of this lane
+    // Start state (h, a mu) of a step that does not continue from registers:
+    // at a segment start the boundary state (h0 for the first) and zero; inside
+    // a long block the checkpoint phase 1 left. Loaded one step ahead.
+    float4 hpf = make_float4(0.f, 0.f, 0.f, 0.f), npf = hpf;
+    auto prefetch_start = [&](int qq, int rr) {
+        if (qq < 0) return;
+        const BwdTile nt = bwd_tile(qq, rr, ntb, SL, L, longb, TT);
+        if (nt.i == 0) {
+            const float *src = nt.ts == 0 ? (a.h0 ? a.h0 + (b * a.D + d) * N + n0 : nullptr)
+                                          : a.boundary + ((b * nblk + nt.ts / K - 1) * a.D + d) * N + n0;
+            hpf = (dvalid && src) ? make_float4(src[0], src[1], src[2], src[3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+            npf = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else if (!nt.ph1 && nt.i < ntb - 1) {
+            hpf = *reinterpret_cast<const float4 *>(ck_base + (nt.i - 1) * ck_stride);
+            npf = *reinterpret_cast<const float4 *>(ck_base + (nt.i - 1) * ck_stride + 4);
+        }
+    };
+    prefetch_start(q, r);
 
     const float4 *dqc = dq + c;
     const float *Bw = Bf + n0;
@@ -248,17 +254,36 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
     for (int s = 0; s < S - 1; ++s) issue(s);
 
 #pragma unroll 1
-    for (int64_t s = 0; s < nsteps; ++s) {
-        int64_t t0, ti, ts; int tlen; bool ph1;
-        tile_of(s, t0, tlen, ph1, ti, ts);
+    for (int s = 0; q >= 0; ++s, advance(q, r)) {
+        const BwdTile tl = bwd_tile(q, r, ntb, SL, L, longb, TT);
+        const int tlen = tl.tlen;
+        const float4 hs = hpf, ns = npf;   // this step's start state, if it takes one
+        {
+            int q2 = q, r2 = r;
+            advance(q2, r2);
+            prefetch_start(q2, r2);
+        }
         cp_async_wait<S - 2>();
         __syncthreads();
-        issue(s + S - 1);
+        issue((s + S - 1) % S);
         const char *st = smem + (s % S) * LY::stage;
         const IO *xs = reinterpret_cast<const IO *>(st);
         const IO *dts = xs + TT * kCh;
         const IO *zs = dts + TT * kCh;
         const IO *dys = zs + TT * kCh;
+
+        // block starts / ends inside the tile (bit e = token e)
+        uint32_t smask = 0, emask = 0;
+        if (longb) {
+            if (tl.tmod == 0) smask = 1u;
+            const int ee = K - 1 - tl.tmod;
+            if (ee < tlen) emask = 1u << ee;
+        } else {
+            for (int e = 0; e < tlen; e += K) {
+                smask |= 1u << e;
+                emask |= 1u << (e + K - 1);
+            }
+        }
 
         // ---- per-element preprocessing: delta, delta*x, ds = dy * gate ----------
         {
@@ -281,129 +306,121 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
         __syncthreads();
 
         // ---- state at the tile start -------------------------------------------
-        if (ti == 0) {
-            init_segment(ts);
-        } else if (!ph1 && ti < ntb - 1) {   // (tile ntb-1 continues from phase 1's registers)
-            const float4 hv = *reinterpret_cast<const float4 *>(ck_base + (ti - 1) * ck_stride);
-            const float4 nv = *reinterpret_cast<const float4 *>(ck_base + (ti - 1) * ck_stride + 4);
-            h[0] = hv.x; h[1] = hv.y; h[2] = hv.z; h[3] = hv.w;
-            nu[0] = nv.x; nu[1] = nv.y; nu[2] = nv.z; nu[3] = nv.w;
+        if (tl.i == 0 || (!tl.ph1 && tl.i < ntb - 1)) {   // (tile ntb-1 continues from phase 1's registers)
+            h2[0] = make_float2(hs.x, hs.y);
+            h2[1] = make_float2(hs.z, hs.w);
+            nu2[0] = make_float2(ns.x, ns.y);
+            nu2[1] = make_float2(ns.z, ns.w);
         }
 
-        if (ph1) {
-            // ---- phase 1: forward over the tile, leaving the next tile's checkpoint
-#pragma unroll
-            for (int t = 0; t < TT; ++t) {
-                if (t < tlen) {
-                    const float4 q4 = dqc[t * kCh];
-                    float at[NPT], bq[NPT];
-                    decay_input<NPT>(al, make_float2(q4.x, q4.y), Bw + t * N, at, bq);
-                    const bool bstart = (t0 + t) % K == 0;
-#pragma unroll
-                    for (int j = 0; j < NPT; ++j) {
-                        const float mu = __fmaf_rn(q4.z, Cw[t * N + j], bstart ? 0.f : nu[j]);
-                        nu[j] = __fmul_rn(at[j], mu);
-                        h[j] = __fmaf_rn(at[j], h[j], bq[j]);
-                    }
-                }
-            }
-            if (ti + 1 < ntb - 1) {
-                float *p = ck_base + ti * ck_stride;
-                *reinterpret_cast<float4 *>(p) = make_float4(h[0], h[1], h[2], h[3]);
-                *reinterpret_cast<float4 *>(p + 4) = make_float4(nu[0], nu[1], nu[2], nu[3]);
-            }
-            continue;
-        }
-
-        // ---- phase 2 (a): forward sweep, per-token a, b, h_{t-1}, mu into TMEM --
+        // ---- forward sweep over the tile (phase 1: state only; phase 2: into TMEM)
 #pragma unroll
         for (int t = 0; t < TT; ++t) {
             if (t < tlen) {
                 const float4 q4 = dqc[t * kCh];
-                float at[NPT], bq[NPT], va[8], vh[8];
+                const float4 Cv = *reinterpret_cast<const float4 *>(Cw + t * N);
+                float at[NPT], bq[NPT];
                 decay_input<NPT>(al, make_float2(q4.x, q4.y), Bw + t * N, at, bq);
-                if ((t0 + t) % K == 0) {
-#pragma unroll
-                    for (int j = 0; j < NPT; ++j) nu[j] = 0.f;
+                if ((smask >> t) & 1u) {
+                    nu2[0] = f2(0.f);
+                    nu2[1] = f2(0.f);
                 }
+                const float2 ds2 = f2(q4.z);
+                const float2 C2[2] = {make_float2(Cv.x, Cv.y), make_float2(Cv.z, Cv.w)};
+                float va[8], vh[8];
 #pragma unroll
-                for (int j = 0; j < NPT; ++j) {
-                    const float mu = __fmaf_rn(q4.z, Cw[t * N + j], nu[j]);
-                    va[j] = at[j];
-                    va[4 + j] = bq[j];
-                    vh[j] = h[j];
-                    vh[4 + j] = mu;
-                    nu[j] = __fmul_rn(at[j], mu);
-                    h[j] = __fmaf_rn(at[j], h[j], bq[j]);
+                for (int p = 0; p < 2; ++p) {
+                    const float2 a2 = make_float2(at[2 * p], at[2 * p + 1]);
+                    const float2 b2 = make_float2(bq[2 * p], bq[2 * p + 1]);
+                    const float2 mu2 = __ffma2_rn(ds2, C2[p], nu2[p]);
+                    va[2 * p] = a2.x; va[2 * p + 1] = a2.y;
+                    va[4 + 2 * p] = b2.x; va[5 + 2 * p] = b2.y;
+                    vh[2 * p] = h2[p].x; vh[2 * p + 1] = h2[p].y;
+                    vh[4 + 2 * p] = mu2.x; vh[5 + 2 * p] = mu2.y;
+                    nu2[p] = __fmul2_rn(a2, mu2);
+                    h2[p] = __ffma2_rn(a2, h2[p], b2);
                 }
-                tmem_st8(tw + t * 16, va);
-                tmem_st8(tw + t * 16 + 8, vh);
+                if (!tl.ph1) {
+                    tmem_st8(tw + t * 16, va);
+                    tmem_st8(tw + t * 16 + 8, vh);
+                }
             }
+        }
+        if (tl.ph1) {
+            if (tl.i + 1 < ntb - 1) {
+                float *p = ck_base + tl.i * ck_stride;
+                *reinterpret_cast<float4 *>(p) = make_float4(h2[0].x, h2[0].y, h2[1].x, h2[1].y);
+                *reinterpret_cast<float4 *>(p + 4) = make_float4(nu2[0].x, nu2[0].y, nu2[1].x, nu2[1].y);
+            }
+            continue;
         }
         tmem_wait_st();
 
-        // ---- phase 2 (b): backward sweep, the adjoint chains --------------------
-        float pq[TT], qq[TT], sq[TT];
-#pragma unroll
-        for (int t = TT - 1; t >= 0; --t) {
-            pq[t] = 0.f;
-            qq[t] = 0.f;
-            sq[t] = 0.f;
-            if (t < tlen) {
-                float va[8], vh[8];
-                tmem_ld8(tw + t * 16, va);
-                tmem_ld8(tw + t * 16 + 8, vh);
-                tmem_wait_ld(va, vh);
-                const float4 q4 = dqc[t * kCh];   // delta, delta*x, ds
-                if ((t0 + t + 1) % K == 0) {
-#pragma unroll
-                    for (int j = 0; j < NPT; ++j) g[j] = 0.f;
-                }
-                float P = 0.f, Q = 0.f, Sg = 0.f, vbc[8];
-#pragma unroll
-                for (int j = 0; j < NPT; ++j) {
-                    const float aj = va[j], bj = va[4 + j], hp = vh[j], mu = vh[4 + j];
-                    const float Cn = Cw[t * N + j], Bn = Bw[t * N + j];
-                    const float lam = __fmaf_rn(q4.z, Cn, rho[j]);
-                    const float db = __fadd_rn(lam, mu);
-                    const float da = __fmaf_rn(mu, g[j], __fmul_rn(lam, hp));
-                    const float gn = __fmaf_rn(aj, g[j], bj);
-                    const float hn = __fmaf_rn(aj, hp, bj);
-                    const float hg = __fadd_rn(hn, gn);
-                    const float qa = __fmul_rn(da, aj);
-                    P = __fmaf_rn(db, Bn, P);
-                    Q = __fmaf_rn(qa, Av[j], Q);
-                    Sg = __fmaf_rn(Cn, hg, Sg);
-                    dAacc[j] = __fmaf_rn(qa, q4.x, dAacc[j]);
-                    vbc[j] = __fmul_rn(db, q4.y);
-                    vbc[4 + j] = __fmul_rn(q4.z, hg);
-                    rho[j] = __fmul_rn(aj, lam);
-                    g[j] = gn;
-                }
-                pq[t] = P;
-                qq[t] = Q;
-                sq[t] = Sg;
-                const float r = lane_reduce_scatter8(vbc, c);
-                if ((c & 3) == 0) {
-                    const int k = c >> 2;
-                    bcs[t * 2 * N + (k < 4 ? n0 + k : N + n0 + k - 4)] = r;
-                }
-            }
-        }
+        // ---- phase 2 backward sweep: the adjoint chains --------------------------
         {
-            float *r0 = red + (warp * kCh + c) * RP;
-            float *r1 = r0 + W * kCh * RP;
-            float *r2 = r1 + W * kCh * RP;
+            float va[8], vh[8];
+            tmem_ld8(tw + (tlen - 1) * 16, va);
+            tmem_ld8(tw + (tlen - 1) * 16 + 8, vh);
+            tmem_wait_ld(va, vh);
+            float *redw = red + (warp * TT) * kCh + c;   // [q][warp][t][lane]
 #pragma unroll
-            for (int q = 0; q < TT / 4; ++q) {
-                *reinterpret_cast<float4 *>(r0 + 4 * q) = make_float4(pq[4 * q], pq[4 * q + 1], pq[4 * q + 2], pq[4 * q + 3]);
-                *reinterpret_cast<float4 *>(r1 + 4 * q) = make_float4(qq[4 * q], qq[4 * q + 1], qq[4 * q + 2], qq[4 * q + 3]);
-                *reinterpret_cast<float4 *>(r2 + 4 * q) = make_float4(sq[4 * q], sq[4 * q + 1], sq[4 * q + 2], sq[4 * q + 3]);
+            for (int t = TT - 1; t >= 0; --t) {
+                if (t < tlen) {
+                    float na[8], nh[8];
+                    if (t > 0) {   // next token's row, read while this one computes
+                        tmem_ld8(tw + (t - 1) * 16, na);
+                        tmem_ld8(tw + (t - 1) * 16 + 8, nh);
+                    }
+                    const float4 q4 = dqc[t * kCh];   // delta, delta*x, ds
+                    const float4 Bv = *reinterpret_cast<const float4 *>(Bw + t * N);
+                    const float4 Cv = *reinterpret_cast<const float4 *>(Cw + t * N);
+                    if ((emask >> t) & 1u) {
+                        g2[0] = f2(0.f);
+                        g2[1] = f2(0.f);
+                    }
+                    const float2 ds2 = f2(q4.z), dl2 = f2(q4.x), dlx2 = f2(q4.y);
+                    const float2 C2[2] = {make_float2(Cv.x, Cv.y), make_float2(Cv.z, Cv.w)};
+                    const float2 B2[2] = {make_float2(Bv.x, Bv.y), make_float2(Bv.z, Bv.w)};
+                    float2 P2 = f2(0.f), Q2 = f2(0.f), S2 = f2(0.f), dB2[2], dC2[2];
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        const float2 a2 = make_float2(va[2 * p], va[2 * p + 1]);
+                        const float2 b2 = make_float2(va[4 + 2 * p], va[5 + 2 * p]);
+                        const float2 hp2 = make_float2(vh[2 * p], vh[2 * p + 1]);
+                        const float2 mu2 = make_float2(vh[4 + 2 * p], vh[5 + 2 * p]);
+                        const float2 lam2 = __ffma2_rn(ds2, C2[p], rho2[p]);
+                        const float2 db2 = __fadd2_rn(lam2, mu2);
+                        const float2 da2 = __ffma2_rn(mu2, g2[p], __fmul2_rn(lam2, hp2));
+                        const float2 gn2 = __ffma2_rn(a2, g2[p], b2);
+                        const float2 hn2 = __ffma2_rn(a2, hp2, b2);
+                        const float2 hg2 = __fadd2_rn(hn2, gn2);
+                        const float2 qa2 = __fmul2_rn(da2, a2);
+                        P2 = __ffma2_rn(db2, B2[p], P2);
+                        Q2 = __ffma2_rn(qa2, Av2[p], Q2);
+                        if (gated) S2 = __ffma2_rn(C2[p], hg2, S2);
+                        dA2[p] = __ffma2_rn(qa2, dl2, dA2[p]);
+                        dB2[p] = __fmul2_rn(db2, dlx2);
+                        dC2[p] = __fmul2_rn(ds2, hg2);
+                        rho2[p] = __fmul2_rn(a2, lam2);
+                        g2[p] = gn2;
+                    }
+                    redw[t * kCh] = __fadd_rn(P2.x, P2.y);
+                    redw[(W * TT + t) * kCh] = __fadd_rn(Q2.x, Q2.y);
+                    if (gated) redw[(2 * W * TT + t) * kCh] = __fadd_rn(S2.x, S2.y);
+                    float *brow = bcr + (t * kCh + c) * BR + n0;
+                    *reinterpret_cast<float4 *>(brow) = make_float4(dB2[0].x, dB2[0].y, dB2[1].x, dB2[1].y);
+                    *reinterpret_cast<float4 *>(brow + N) = make_float4(dC2[0].x, dC2[0].y, dC2[1].x, dC2[1].y);
+                    if (t > 0) {
+                        tmem_wait_ld(na, nh);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) { va[j] = na[j]; vh[j] = nh[j]; }
+                    }
+                }
             }
         }
         __syncthreads();
 
-        // ---- readout: dx, d(dt), dz of the tile; dB | dC partial rows ------------
+        // ---- readout: dx, d(dt), dz of the tile's (token, channel) pairs ---------
         if (warp * PER < TT) {
 #pragma unroll
             for (int i = 0; i < PER; ++i) {
@@ -412,10 +429,10 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
                     float P = 0.f, Q = 0.f, Sg = 0.f;
 #pragma unroll
                     for (int gg = 0; gg < W; ++gg) {
-                        const float *rr = red + (gg * kCh + c) * RP + t;
+                        const float *rr = red + (gg * TT + t) * kCh + c;
                         P = __fadd_rn(P, rr[0]);
-                        Q = __fadd_rn(Q, rr[W * kCh * RP]);
-                        Sg = __fadd_rn(Sg, rr[2 * W * kCh * RP]);
+                        Q = __fadd_rn(Q, rr[W * TT * kCh]);
+                        if (gated) Sg = __fadd_rn(Sg, rr[2 * W * TT * kCh]);
                     }
                     const int e = t * kCh + c;
                     const float4 q4 = dq[e];
@@ -423,7 +440,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
                     const float dxv = __fmaf_rn(q4.x, P, __fmul_rn(dfac, q4.z));
                     float ddl = __fmaf_rn(xv, P, Q);
                     if (a.dt_softplus) ddl = __fmul_rn(ddl, sigmoid_f32(to_f32(dts[e])));
-                    const int64_t go = (b * L + t0 + t) * a.D + d;
+                    const int64_t go = (b * L + tl.t0 + t) * a.D + d;
                     IO o;
                     from_f32(dxv, o);
                     static_cast<IO *>(a.dx)[go] = o;
@@ -441,10 +458,36 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
                 }
             }
         }
+        // ---- dB | dC of the tile summed over the CTA's 32 channels: one row per
+        // token. Two threads per float4 group, 16 lanes each, then one exchange.
         {
-            float *dst = a.ws_bc + ((b * CT + ct) * L + t0) * 2 * N;
-            for (int e = tid; e < tlen * 2 * N / 4; e += NT)
-                reinterpret_cast<float4 *>(dst)[e] = reinterpret_cast<const float4 *>(bcs)[e];
+            constexpr int G4 = 2 * N / 4;   // float4 groups per row
+            float4 *dst = reinterpret_cast<float4 *>(a.ws_bc + ((b * CT + ct) * L + tl.t0) * 2 * N);
+            const int ntask = tlen * G4;
+            for (int k2 = tid; k2 < ((ntask * 2 + 31) & ~31); k2 += NT) {   // whole warps (shuffle)
+                const int k = k2 >> 1, half = k2 & 1;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (k < ntask) {
+                    const int t = k / G4, j4 = k % G4;
+                    const float *src = bcr + (t * kCh + half * 16) * BR + j4 * 4;
+#pragma unroll 8
+                    for (int l = 0; l < 16; ++l) {   // the two halves start 8 lanes apart: no bank clash
+                        const float4 v = *reinterpret_cast<const float4 *>(src + ((l + half * 8) & 15) * BR);
+                        acc.x = __fadd_rn(acc.x, v.x);
+                        acc.y = __fadd_rn(acc.y, v.y);
+                        acc.z = __fadd_rn(acc.z, v.z);
+                        acc.w = __fadd_rn(acc.w, v.w);
+                    }
+                }
+                float4 o;
+                o.x = __shfl_xor_sync(0xffffffffu, acc.x, 1);
+                o.y = __shfl_xor_sync(0xffffffffu, acc.y, 1);
+                o.z = __shfl_xor_sync(0xffffffffu, acc.z, 1);
+                o.w = __shfl_xor_sync(0xffffffffu, acc.w, 1);
+                if (k < ntask && half == 0)
+                    dst[k] = make_float4(__fadd_rn(acc.x, o.x), __fadd_rn(acc.y, o.y), __fadd_rn(acc.z, o.z),
+                                         __fadd_rn(acc.w, o.w));
+            }
         }
     }
     cp_async_wait<0>();
@@ -455,9 +498,13 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
 
     if (dvalid) {
 #pragma unroll
-        for (int j = 0; j < NPT; ++j) {
-            if (a.dh0) a.dh0[(b * a.D + d) * N + n0 + j] = rho[j];
-            a.ws_a[(b * a.D + d) * N + n0 + j] = dAacc[j];
+        for (int p = 0; p < 2; ++p) {
+            if (a.dh0) {
+                a.dh0[(b * a.D + d) * N + n0 + 2 * p] = rho2[p].x;
+                a.dh0[(b * a.D + d) * N + n0 + 2 * p + 1] = rho2[p].y;
+            }
+            a.ws_a[(b * a.D + d) * N + n0 + 2 * p] = dA2[p].x;
+            a.ws_a[(b * a.D + d) * N + n0 + 2 * p + 1] = dA2[p].y;
         }
     }
     dsk[warp * kCh + c] = dskacc;
