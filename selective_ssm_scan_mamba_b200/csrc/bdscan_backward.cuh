@@ -227,24 +227,15 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
     };
     float *ck_base = a.ws_ck ? a.ws_ck + (((b * CT + ct) * a.nck * W + warp) * kCh + c) * 8 : nullptr;
     const int64_t ck_stride = (int64_t)W * kCh * 8;   // between consecutive checkpoints of this lane
-    // Start state (h, a mu) of a step that does not continue from registers:
-    // at a segment start the boundary state (h0 for the first) and zero; inside
-    // a long block the checkpoint phase 1 left. Loaded one step ahead.
-    float4 hpf = make_float4(0.f, 0.f, 0.f, 0.f), npf = hpf;
-    auto prefetch_start = [&](int qq, int rr) {
-        if (qq < 0) return;
-        const BwdTile nt = bwd_tile(qq, rr, ntb, SL, L, longb, TT);
-        if (nt.i == 0) {
-            const float *src = nt.ts == 0 ? (a.h0 ? a.h0 + (b * a.D + d) * N + n0 : nullptr)
-                                          : a.boundary + ((b * nblk + nt.ts / K - 1) * a.D + d) * N + n0;
-            hpf = (dvalid && src) ? make_float4(src[0], src[1], src[2], src[3]) : make_float4(0.f, 0.f, 0.f, 0.f);
-            npf = make_float4(0.f, 0.f, 0.f, 0.f);
-        } else if (!nt.ph1 && nt.i < ntb - 1) {
-            hpf = *reinterpret_cast<const float4 *>(ck_base + (nt.i - 1) * ck_stride);
-            npf = *reinterpret_cast<const float4 *>(ck_base + (nt.i - 1) * ck_stride + 4);
+    auto init_segment = [&](int64_t ts) {   // forward state at a block start, reverse adjoint zero
+        const float *src = ts == 0 ? (a.h0 ? a.h0 + (b * a.D + d) * N + n0 : nullptr)
+                                   : a.boundary + ((b * nblk + ts / K - 1) * a.D + d) * N + n0;
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            h2[p] = (dvalid && src) ? make_float2(src[2 * p], src[2 * p + 1]) : f2(0.f);
+            nu2[p] = f2(0.f);
         }
     };
-    prefetch_start(q, r);
 
     const float4 *dqc = dq + c;
     const float *Bw = Bf + n0;
@@ -257,12 +248,6 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
     for (int s = 0; q >= 0; ++s, advance(q, r)) {
         const BwdTile tl = bwd_tile(q, r, ntb, SL, L, longb, TT);
         const int tlen = tl.tlen;
-        const float4 hs = hpf, ns = npf;   // this step's start state, if it takes one
-        {
-            int q2 = q, r2 = r;
-            advance(q2, r2);
-            prefetch_start(q2, r2);
-        }
         cp_async_wait<S - 2>();
         __syncthreads();
         issue((s + S - 1) % S);
@@ -306,11 +291,15 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
         __syncthreads();
 
         // ---- state at the tile start -------------------------------------------
-        if (tl.i == 0 || (!tl.ph1 && tl.i < ntb - 1)) {   // (tile ntb-1 continues from phase 1's registers)
-            h2[0] = make_float2(hs.x, hs.y);
-            h2[1] = make_float2(hs.z, hs.w);
-            nu2[0] = make_float2(ns.x, ns.y);
-            nu2[1] = make_float2(ns.z, ns.w);
+        if (tl.i == 0) {
+            init_segment(tl.ts);
+        } else if (!tl.ph1 && tl.i < ntb - 1) {   // (tile ntb-1 continues from phase 1's registers)
+            const float4 hv = *reinterpret_cast<const float4 *>(ck_base + (tl.i - 1) * ck_stride);
+            const float4 nv = *reinterpret_cast<const float4 *>(ck_base + (tl.i - 1) * ck_stride + 4);
+            h2[0] = make_float2(hv.x, hv.y);
+            h2[1] = make_float2(hv.z, hv.w);
+            nu2[0] = make_float2(nv.x, nv.y);
+            nu2[1] = make_float2(nv.z, nv.w);
         }
 
         // ---- forward sweep over the tile (phase 1: state only; phase 2: into TMEM)
@@ -458,35 +447,22 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
                 }
             }
         }
-        // ---- dB | dC of the tile summed over the CTA's 32 channels: one row per
-        // token. Two threads per float4 group, 16 lanes each, then one exchange.
+        // ---- dB | dC of the tile summed over the CTA's 32 channels: one row per token
         {
             constexpr int G4 = 2 * N / 4;   // float4 groups per row
             float4 *dst = reinterpret_cast<float4 *>(a.ws_bc + ((b * CT + ct) * L + tl.t0) * 2 * N);
-            const int ntask = tlen * G4;
-            for (int k2 = tid; k2 < ((ntask * 2 + 31) & ~31); k2 += NT) {   // whole warps (shuffle)
-                const int k = k2 >> 1, half = k2 & 1;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (k < ntask) {
-                    const int t = k / G4, j4 = k % G4;
-                    const float *src = bcr + (t * kCh + half * 16) * BR + j4 * 4;
+            for (int k = tid; k < tlen * G4; k += NT) {
+                const int t = k / G4, j4 = k % G4;
+                const float *src = bcr + t * kCh * BR + j4 * 4;
+                const float4 v0 = *reinterpret_cast<const float4 *>(src);
+                float2 lo = make_float2(v0.x, v0.y), hi = make_float2(v0.z, v0.w);
 #pragma unroll 8
-                    for (int l = 0; l < 16; ++l) {   // the two halves start 8 lanes apart: no bank clash
-                        const float4 v = *reinterpret_cast<const float4 *>(src + ((l + half * 8) & 15) * BR);
-                        acc.x = __fadd_rn(acc.x, v.x);
-                        acc.y = __fadd_rn(acc.y, v.y);
-                        acc.z = __fadd_rn(acc.z, v.z);
-                        acc.w = __fadd_rn(acc.w, v.w);
-                    }
+                for (int l = 1; l < kCh; ++l) {
+                    const float4 v = *reinterpret_cast<const float4 *>(src + l * BR);
+                    lo = __fadd2_rn(lo, make_float2(v.x, v.y));
+                    hi = __fadd2_rn(hi, make_float2(v.z, v.w));
                 }
-                float4 o;
-                o.x = __shfl_xor_sync(0xffffffffu, acc.x, 1);
-                o.y = __shfl_xor_sync(0xffffffffu, acc.y, 1);
-                o.z = __shfl_xor_sync(0xffffffffu, acc.z, 1);
-                o.w = __shfl_xor_sync(0xffffffffu, acc.w, 1);
-                if (k < ntask && half == 0)
-                    dst[k] = make_float4(__fadd_rn(acc.x, o.x), __fadd_rn(acc.y, o.y), __fadd_rn(acc.z, o.z),
-                                         __fadd_rn(acc.w, o.w));
+                dst[k] = make_float4(lo.x, lo.y, hi.x, hi.y);
             }
         }
     }

@@ -628,10 +628,12 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
 #pragma unroll
                     for (int q = 0; q < PER / 4; ++q) {
                         const float4 v = *reinterpret_cast<const float4 *>(rrow + 4 * q);
-                        ysum[4 * q] = __fadd_rn(ysum[4 * q], v.x);
-                        ysum[4 * q + 1] = __fadd_rn(ysum[4 * q + 1], v.y);
-                        ysum[4 * q + 2] = __fadd_rn(ysum[4 * q + 2], v.z);
-                        ysum[4 * q + 3] = __fadd_rn(ysum[4 * q + 3], v.w);
+                        const float2 s0 = __fadd2_rn(make_float2(ysum[4 * q], ysum[4 * q + 1]), make_float2(v.x, v.y));
+                        const float2 s1 = __fadd2_rn(make_float2(ysum[4 * q + 2], ysum[4 * q + 3]), make_float2(v.z, v.w));
+                        ysum[4 * q] = s0.x;
+                        ysum[4 * q + 1] = s0.y;
+                        ysum[4 * q + 2] = s1.x;
+                        ysum[4 * q + 3] = s1.y;
                     }
                 } else {
 #pragma unroll
