@@ -39,11 +39,27 @@ int check_common(const bdscan_dims *dm, const bdscan_inputs *in) {
     return BDSCAN_OK;
 }
 
+// dynamic shared memory a CTA may opt in to on sm_100 (227 KB), less room for the
+// kernels' static shared memory
+constexpr int kMaxDynSmem = 226 * 1024;
+
+// span checkpoints of the long fused path: (spans - 1) x N states x 32 channels, fp32
+size_t long_fused_ck_bytes(int64_t K, int N) {
+    const int64_t spans = (K + bdk::kSpanLong - 1) / bdk::kSpanLong;
+    return (size_t)(spans - 1) * (size_t)N * bdk::kCh * 4;
+}
+
+template <class IO, int N>
+bool long_fused_fits(int64_t K) {
+    return bdk::Layout<IO, N, bdk::kLongFused, 0>::base_bytes + long_fused_ck_bytes(K, N) <= (size_t)kMaxDynSmem;
+}
+
 template <class IO, int N, int MODE, int KC>
 int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1) {
     using CF = bdk::Cfg<N, MODE, KC>;
     using LY = bdk::Layout<IO, N, MODE, KC>;
-    const size_t smem = LY::base_bytes + (MODE == bdk::kLong ? (size_t)a.K * bdk::kCh * 4 : 0);
+    const size_t smem = LY::base_bytes + (MODE == bdk::kLong ? (size_t)a.K * bdk::kCh * 4
+                                          : MODE == bdk::kLongFused ? long_fused_ck_bytes(a.K, N) : 0);
     auto kern = bdk::bdscan_kernel<IO, N, MODE, KC>;
     // raise the dynamic shared-memory ceiling once per device
     static std::atomic<uint64_t> done_mask{0};
@@ -51,7 +67,8 @@ int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz =
     if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
     const uint64_t bit = 1ull << (dev & 63);
     if (!(done_mask.load(std::memory_order_acquire) & bit)) {
-        const int cap = LY::base_bytes + (MODE == bdk::kLong ? bdk::kLongSmemMax : 0);
+        const int cap = MODE == bdk::kLongFused ? kMaxDynSmem
+                                                 : LY::base_bytes + (MODE == bdk::kLong ? bdk::kLongSmemMax : 0);
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
         if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
         done_mask.fetch_or(bit, std::memory_order_acq_rel);
@@ -67,6 +84,7 @@ template <class IO, int N>
 int dispatch_mode(int mode, const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1) {
     if (mode == bdk::kForwardOnly) return launch<IO, N, bdk::kForwardOnly, 0>(a, batch, st, gz);
     if (mode == bdk::kLong) return launch<IO, N, bdk::kLong, 0>(a, batch, st);
+    if (mode == bdk::kLongFused) return launch<IO, N, bdk::kLongFused, 0>(a, batch, st);
     if (mode == bdk::kReverseAcc) return launch<IO, N, bdk::kReverseAcc, 0>(a, batch, st);
     switch (a.K) {
         case 4: return launch<IO, N, bdk::kFused, 4>(a, batch, st);
@@ -104,8 +122,17 @@ int run(Op op, const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, 
     } else if (dm->block <= 32) {
         mode = bdk::kFused;
     } else {
-        if (dm->block * bdk::kCh * 4 > bdk::kLongSmemMax) return BDSCAN_ERR_UNSUPPORTED;
-        mode = bdk::kLong;
+        const bool bf = dm->io_dtype == BDSCAN_BF16;
+        const bool fits = dm->d_state == 16 ? (bf ? long_fused_fits<__nv_bfloat16, 16>(dm->block)
+                                                  : long_fused_fits<float, 16>(dm->block))
+                                            : (bf ? long_fused_fits<__nv_bfloat16, 64>(dm->block)
+                                                  : long_fused_fits<float, 64>(dm->block));
+        if (fits) {
+            mode = bdk::kLongFused;
+        } else {
+            if (dm->block * bdk::kCh * 4 > bdk::kLongSmemMax) return BDSCAN_ERR_UNSUPPORTED;
+            mode = bdk::kLong;
+        }
     }
     if (dm->batch == 0 || dm->d_inner == 0) return BDSCAN_OK;   // nothing to compute or write
 

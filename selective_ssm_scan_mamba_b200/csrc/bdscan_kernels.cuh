@@ -37,7 +37,13 @@
 //            whole sequence, tiles last to first, adding y_rev + Dskip x to the
 //            forward pass's y in place and applying the gate.
 //   long   = blocks longer than 32 tokens: per block, a reverse sweep over its
-//            tiles from last to first (carrying g) whose readout is staged in
+//            16-token spans from last to first that carries only the reverse
+//            state g and leaves it in shared memory at every span start (the
+//            span's right-hand boundary condition); then the forward sweep runs
+//            the whole-block fused pattern span by span (TMEM, interleaved
+//            chains), each span's reverse chain starting from its checkpoint.
+//            Blocks whose checkpoints do not fit in shared memory take the
+//            older two-sweep path: a reverse sweep whose readout is staged in
 //            shared memory, then a forward sweep that adds it (two exps per
 //            element).
 #pragma once
@@ -47,9 +53,10 @@
 namespace bdk {
 
 constexpr int kCh = 32;                  // channels per CTA (one per lane)
-constexpr int kLongSmemMax = 96 * 1024;  // y_rev staging limit of the long-block path
+constexpr int kLongSmemMax = 96 * 1024;  // y_rev staging limit of the two-sweep long-block path
+constexpr int kSpanLong = 16;            // span of the checkpointed long-block path
 
-enum Mode { kForwardOnly = 0, kFused = 1, kLong = 2, kReverseAcc = 3 };
+enum Mode { kForwardOnly = 0, kFused = 1, kLong = 2, kReverseAcc = 3, kLongFused = 4 };
 
 struct ScanArgs {
     const void *x, *dt, *B, *C, *z;
@@ -85,7 +92,8 @@ struct Cfg {
     static constexpr int NPT = Npt<N, MODE>::value;
     static constexpr int W = N / NPT;                 // warps per CTA (state groups)
     static constexpr int THREADS = 32 * W;
-    static constexpr int T = (MODE == kFused && (KC == 0 || KC > 16 || (KC == 16 && N == 16))) ? 32 : 16;   // tokens per tile
+    static constexpr int T = (MODE == kFused && (KC == 0 || KC > 16 || (KC == 16 && N == 16))) ? 32
+                             : ((MODE == kLongFused && N == 16) ? 32 : 16);   // tokens per tile
     static constexpr int S = T == 16 ? 4 : 3;                                    // cp.async ring depth
     static constexpr int SPAN = MODE == kFused ? (KC > 0 ? KC : T) : 16;
     static constexpr bool KEEP_B = SPAN <= 16 && N == 16;                        // keep b for phase C
@@ -96,12 +104,13 @@ struct Cfg {
     // the largest residency these variants reach (N = 16, K = 32: 2 CTAs x 256).
     static constexpr int WCOLS = SPAN * 2 * NPT;
     static constexpr int TNEED = (W / 4) * WCOLS;
-    static constexpr bool TMEM = MODE == kFused && KC > 0 && W % 4 == 0 && NPT == 4 && TNEED <= 512;
+    static constexpr bool TMEM = ((MODE == kFused && KC > 0) || MODE == kLongFused) && W % 4 == 0 && NPT == 4 &&
+                                 TNEED <= 512;
     static constexpr int TCOLS = TNEED <= 32 ? 32 : (TNEED <= 64 ? 64 : (TNEED <= 128 ? 128 : (TNEED <= 256 ? 256 : 512)));
     // registers: the four N = 16 state-group warps of a CTA sit on the SM's four
     // sub-partitions, so 3 resident CTAs = 3 warps per sub-partition (<= 168
     // registers), enough for a 12288-channel batch in one wave on 148 SMs.
-    static constexpr int MINB = THREADS >= 512 ? 1 : ((T == 16 || KC == 16) ? 3 : 2);
+    static constexpr int MINB = THREADS >= 512 ? 1 : ((T == 16 || KC == 16 || MODE == kLongFused) ? 3 : 2);
     static_assert(N % NPT == 0 && W <= 32, "state split");
 };
 
@@ -118,7 +127,8 @@ struct Layout {
     static constexpr int bf = dd + T * kCh * 8;            // float B                  [T][N]
     static constexpr int cf = bf + T * N * 4;              // float C                  [T][N]
     static constexpr int red = cf + T * N * 4;             // float partial readouts   [W][32][RP]
-    static constexpr int yrev = red + W * kCh * RP * 4;    // float reverse readout    [K][32] (long)
+    static constexpr int yrev = red + W * kCh * RP * 4;    // float reverse readout [K][32] (long), or the
+                                                           // float4 span checkpoints [spans-1][W][32] (long fused)
     static constexpr int base_bytes = yrev;
     static_assert(xb % 16 == 0 && bb % 16 == 0 && (RP * 4) % 16 == 0, "16-byte rows");
 };
@@ -301,10 +311,28 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
     // forward-only / fused: step s covers tokens [s*TE, min((s+1)*TE, L)).
     // long: per block j, nt reverse steps (tiles nt-1 .. 0) then nt forward steps.
     const int TE = (MODE == kFused && KC == 0) ? (int)((T / K) * K) : T;
-    const int64_t nt_blk = (MODE == kLong) ? (K + T - 1) / T : 1;
-    const int64_t nsteps = (MODE == kLong) ? (L / K) * 2 * nt_blk : (tend - tbeg + TE - 1) / TE;   // kReverseAcc: TE = T
+    constexpr bool LONGM = MODE == kLong || MODE == kLongFused;
+    const int64_t nt_blk = LONGM ? (K + T - 1) / T : 1;
+    // long fused: reverse steps cover every tile but the first, plus the first
+    // tile's second span when a tile holds two spans
+    const int64_t nr_blk = MODE == kLongFused ? (T == SPAN ? nt_blk - 1 : nt_blk) : nt_blk;
+    const int64_t nsteps = MODE == kLong ? (L / K) * 2 * nt_blk
+                         : MODE == kLongFused ? (L / K) * (nr_blk + nt_blk)
+                                              : (tend - tbeg + TE - 1) / TE;   // kReverseAcc: TE = T
+    const int nspan = MODE == kLongFused ? (int)((K + SPAN - 1) / SPAN) : 1;   // spans per block
+    int64_t tile_in_blk = 0;   // long modes: index of the current tile inside its block
     auto tile_of = [&](int64_t s, int64_t &t0, int &tlen, bool &rev, bool &first_rev) {
-        if (MODE == kLong) {
+        if (MODE == kLongFused) {
+            const int64_t per = nr_blk + nt_blk;
+            const int64_t j = s / per, r = s % per;
+            rev = r < nr_blk;
+            const int64_t i = rev ? nt_blk - 1 - r : r - nr_blk;
+            first_rev = rev && r == 0;
+            tile_in_blk = i;
+            t0 = j * K + i * T;
+            const int64_t rem = (j + 1) * K - t0;
+            tlen = (int)(rem < T ? rem : T);
+        } else if (MODE == kLong) {
             const int64_t j = s / (2 * nt_blk), r = s % (2 * nt_blk);
             rev = r < nt_blk;
             const int64_t i = rev ? nt_blk - 1 - r : r - nt_blk;
@@ -367,6 +395,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
     for (int64_t s = 0; s < nsteps; ++s) {
         int64_t t0; int tlen; bool rev, first_rev;
         tile_of(s, t0, tlen, rev, first_rev);
+        const int64_t ti = tile_in_blk;   // (issue() below reuses tile_of)
         cp_async_wait<S - 2>();
         __syncthreads();   // stage s landed for every thread; step s-1 is fully done
         issue(s + S - 1);
@@ -382,7 +411,8 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
             for (int e = tid; e < T * kCh; e += NT) {
                 const float xv = to_f32(xs[e]);
                 const float dr = to_f32(dts[e]);
-                const float dl = a.dt_softplus ? softplus_f32(dr) : dr;
+                float dl = a.dt_softplus ? softplus_f32(dr) : dr;
+                if (MODE == kLongFused && e / kCh >= tlen) dl = 0.f;   // rows past the block: a = 1, b = 0
                 dd[e] = make_float2(dl, __fmul_rn(dl, xv));
             }
             constexpr int EPC = 16 / (int)sizeof(IO);
@@ -403,6 +433,36 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
         }
 
         if (MODE == kLong && !rev && a.blk_h0 && t0 % K == 0) restart_h(t0 / K);
+
+        if (MODE == kLongFused && rev) {
+            // reverse-state sweep: g only, no readout; at a span's first token g
+            // is the boundary condition of the span before it
+            if (first_rev) {
+#pragma unroll
+                for (int j = 0; j < NPT; ++j) gcar[j] = 0.f;
+            }
+            const int lo = (T > SPAN && ti == 0) ? SPAN : 0;   // the block's first span needs no checkpoint
+            float4 *ck = reinterpret_cast<float4 *>(yrev) + warp * kCh + c;
+            const int sb = (int)ti * (T / SPAN);   // span index of the tile's first token
+#pragma unroll
+            for (int t = T - 1; t >= 0; --t) {
+                if (t >= lo) {
+                    float at[NPT], bq[NPT];
+                    decay_input<NPT>(al, ddc[t * kCh], Bw + t * N, at, bq);
+#pragma unroll
+                    for (int p = 0; p < NPT / 2; ++p) {
+                        const float2 g2 = __ffma2_rn(make_float2(at[2 * p], at[2 * p + 1]),
+                                                     make_float2(gcar[2 * p], gcar[2 * p + 1]),
+                                                     make_float2(bq[2 * p], bq[2 * p + 1]));
+                        gcar[2 * p] = g2.x;
+                        gcar[2 * p + 1] = g2.y;
+                    }
+                    if (t % SPAN == 0 && t < tlen && sb + t / SPAN >= 1)
+                        ck[(int64_t)(sb + t / SPAN - 1) * W * kCh] = make_float4(gcar[0], gcar[1], gcar[2], gcar[3]);
+                }
+            }
+            continue;   // no output from this sweep
+        }
 
         if ((MODE == kLong || MODE == kReverseAcc) && rev) {   // reverse sweep tile: decays, then the chain
             float at[T][NPT];
@@ -425,7 +485,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
                 }
                 yp[t] = acc;
             }
-        } else if (MODE == kFused && KC > 0) {
+        } else if ((MODE == kFused && KC > 0) || MODE == kLongFused) {
             // Whole blocks (a tile holds whole blocks, since L % K == 0 and K
             // divides T): phase A for the block, then the forward and the
             // reverse chains interleaved -- they share only the kept decays, so
@@ -439,10 +499,17 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
                     for (int i = 0; i < SPAN; ++i) yp[s0 + i] = 0.f;
                     continue;
                 }
-                if (a.blk_h0) restart_h((t0 + s0) / K);
+                if (a.blk_h0 && (MODE != kLongFused || (ti == 0 && sp == 0))) restart_h((t0 + s0) / K);
                 float gs[NPT];
 #pragma unroll
                 for (int j = 0; j < NPT; ++j) gs[j] = 0.f;
+                if (MODE == kLongFused) {   // the span's right-hand boundary condition
+                    const int span = (int)ti * (T / SPAN) + sp;
+                    if (span < nspan - 1) {
+                        const float4 g4 = reinterpret_cast<const float4 *>(yrev)[(int64_t)span * W * kCh + warp * kCh + c];
+                        gs[0] = g4.x; gs[1] = g4.y; gs[2] = g4.z; gs[3] = g4.w;
+                    }
+                }
                 if constexpr (CF::TMEM) {
                     // (A) a and b of every token of the block into this warp's TMEM lanes
 #pragma unroll
@@ -523,7 +590,11 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
                         }
                     }
                 }
-                write_boundary(t0 + s0 + SPAN - 1);
+                if (MODE != kLongFused) {
+                    write_boundary(t0 + s0 + SPAN - 1);
+                } else if (s0 + SPAN >= tlen && ti == nt_blk - 1) {
+                    write_boundary(t0 + tlen - 1);   // the span holding the block's last token
+                }
             }
         } else if (MODE == kForwardOnly && chunked && a.chunk_pass == 1) {
             // time-chunked pass 1: the chunk's state from zero and the product of its decays
