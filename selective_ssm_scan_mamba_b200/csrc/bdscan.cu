@@ -127,7 +127,7 @@ int run(Op op, const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, 
                                                   : long_fused_fits<float, 16>(dm->block))
                                             : (bf ? long_fused_fits<__nv_bfloat16, 64>(dm->block)
                                                   : long_fused_fits<float, 64>(dm->block));
-        if (fits) {
+        if (fits && dm->seqlen < (int64_t(1) << 30)) {   // (its tile schedule counts steps in 32 bits)
             mode = bdk::kLongFused;
         } else {
             if (dm->block * bdk::kCh * 4 > bdk::kLongSmemMax) return BDSCAN_ERR_UNSUPPORTED;

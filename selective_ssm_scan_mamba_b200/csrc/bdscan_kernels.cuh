@@ -199,9 +199,10 @@ __device__ __forceinline__ float scan_step(float (&st)[NPT], const float (&a)[NP
 
 // Copy tokens [t0, t0 + tlen) of one CTA's tile into a ring stage; rows past
 // tlen and channels past D are zero-filled without reading global memory.
+// want_c = false leaves C (and z) out: a sweep that carries only the state.
 template <class IO, int N, int T, int NT>
 __device__ __forceinline__ void stage_tile(char *st, const ScanArgs &a, int64_t b, int64_t d0, int64_t t0,
-                                           int tlen, bool gated) {
+                                           int tlen, bool gated, bool want_c = true) {
     constexpr int EPC = 16 / (int)sizeof(IO);   // elements per 16-byte chunk
     constexpr int XC = kCh / EPC;               // chunks per x row
     constexpr int BC = N / EPC;                 // chunks per B row
@@ -227,7 +228,7 @@ __device__ __forceinline__ void stage_tile(char *st, const ScanArgs &a, int64_t 
         const int64_t off = ok ? ((row0 + t) * N + (int64_t)ch * EPC) : 0;
         const int so = t * N + ch * EPC;
         cp_async16(Bs + so, static_cast<const IO *>(a.B) + off, ok);
-        cp_async16(Cs + so, static_cast<const IO *>(a.C) + off, ok);
+        if (want_c) cp_async16(Cs + so, static_cast<const IO *>(a.C) + off, ok);
     }
 }
 
@@ -323,8 +324,8 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
     int64_t tile_in_blk = 0;   // long modes: index of the current tile inside its block
     auto tile_of = [&](int64_t s, int64_t &t0, int &tlen, bool &rev, bool &first_rev) {
         if (MODE == kLongFused) {
-            const int64_t per = nr_blk + nt_blk;
-            const int64_t j = s / per, r = s % per;
+            const int per = (int)(nr_blk + nt_blk);
+            const int j = (int)s / per, r = (int)s - j * per;   // 32-bit: steps < 2^31
             rev = r < nr_blk;
             const int64_t i = rev ? nt_blk - 1 - r : r - nr_blk;
             first_rev = rev && r == 0;
@@ -359,7 +360,9 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::M
         if (s < nsteps) {
             int64_t t0; int tlen; bool rv, fr;
             tile_of(s, t0, tlen, rv, fr);
-            stage_tile<IO, N, T, NT>(smem + (s % S) * LY::stage, a, b, d0, t0, tlen, gated);
+            const bool state_only = MODE == kLongFused && rv;   // the g-only reverse sweep reads no C, z
+            stage_tile<IO, N, T, NT>(smem + (s % S) * LY::stage, a, b, d0, t0, tlen, gated && !state_only,
+                                     !state_only);
         }
         cp_async_commit();
     };

@@ -31,6 +31,8 @@ CASES = [   # (Bt, L, D, N, K, io, gated, h0)
     (1, 96, 32, 16, 48, "f32", True, True),
     (2, 64, 24, 64, 16, "bf16", False, True),
     (1, 64, 16, 64, 4, "f32", True, False),
+    (1, 128, 32, 64, 64, "bf16", True, True),
+    (1, 512, 16, 64, 512, "bf16", False, True),
 ]
 
 
