@@ -93,3 +93,37 @@ def test_cpu_tensors_are_refused_without_fallback():
     t = tensors()
     with pytest.raises(ValueError, match="CUDA"):
         bdscan.train_blocks(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], 16)
+
+
+def test_backward_marshalling(fake):
+    t = tensors()
+    z = torch.zeros(2, 32, 64, dtype=torch.bfloat16)
+    dy = torch.zeros(2, 32, 64, dtype=torch.bfloat16)
+    bnd = torch.zeros(2, 2, 64, 16)
+    h0 = torch.zeros(2, 64, 16)
+    g = bdscan.train_blocks_backward(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], 16, dy, bnd, z=z, h0=h0)
+    name, args = fake.calls[-1]
+    assert name == "bdscan_train_blocks_backward"
+    assert args[2] == h0.data_ptr() and args[3] == bnd.data_ptr() and args[4] == dy.data_ptr()
+    gr = ct.cast(args[5], ct.POINTER(bdscan.Grads)).contents
+    for k in ("dx", "ddt", "dz", "dB", "dC", "dA", "dDskip", "dh0"):
+        assert getattr(gr, k) == g[k].data_ptr(), k
+    assert g["dx"].dtype == torch.bfloat16 and g["dA"].dtype == torch.float32 and g["dB"].shape == (2, 32, 16)
+    assert args[8] == 1234
+    # no gate: no dz output and a NULL pointer for it
+    g2 = bdscan.train_blocks_backward(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], 16, dy, bnd,
+                                      want_dh0=False)
+    gr2 = ct.cast(fake.calls[-1][1][5], ct.POINTER(bdscan.Grads)).contents
+    assert g2["dz"] is None and gr2.dz is None and g2["dh0"] is None and gr2.dh0 is None
+
+
+def test_noalloc_prefill_needs_caller_outputs(fake):
+    t = tensors()
+    y = torch.zeros(2, 32, 64, dtype=torch.bfloat16)
+    h = torch.zeros(2, 64, 16)
+    bdscan.prefill_chunked_noalloc(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], 16, y, h)
+    name, args = fake.calls[-1]
+    assert name == "bdscan_prefill_chunked_noalloc"
+    assert args[3] == y.data_ptr() and args[4] == h.data_ptr() and args[5] is None and args[6] == 1234
+    with pytest.raises(ValueError):   # outputs are checked like inputs
+        bdscan.prefill_chunked_noalloc(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], 16, y[:, :16], h)
