@@ -662,6 +662,76 @@ def run_train_step(args):
     return 0
 
 
+def run_context_parallel(args):
+    """Prefill of the 262,144-token context (batch 4, 2048 channels) split over
+    the ranks (torchrun, one rank per GPU): each rank generates and holds its
+    consecutive chunk, computes its summary, joins one all-gather, folds its
+    start state and prefills its chunk. Time: max over ranks."""
+    import datetime
+    import statistics as st_
+    import torch
+    import torch.distributed as dist
+    from selective_ssm_scan_mamba_b200 import bdscan, context_parallel as cp
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29511")
+        dist.init_process_group("nccl", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    w = I.WORKLOADS["step262k"]
+    K = w.K
+    nblk = w.L // K
+    b0, b1 = rank * nblk // world, (rank + 1) * nblk // world
+    t0, n = b0 * K, (b1 - b0) * K
+
+    def up(a):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.to(dev)
+
+    p = I.make_params(w.seed, w.D, w.N)
+    A, Dk = up(p["A"]), up(p["Dskip"])
+    ctx = {k: torch.empty((w.batch, n, w.D if k in ("x", "dt") else w.N), dtype=torch.bfloat16, device=dev)
+           for k in ("x", "dt", "B", "C")}
+    for c0 in range(0, n, 8 * I.CHUNK):
+        m = min(8 * I.CHUNK, n - c0)
+        sq = I.make_sequence(w.seed, w.batch, m, w.D, w.N, w.io, stream=("context",), t0=t0 + c0)
+        for k in ctx:
+            ctx[k][:, c0:c0 + m] = up(sq[k])
+
+    def step():
+        return cp.prefill_context_parallel(ctx["x"], ctx["dt"], A, ctx["B"], ctx["C"], Dk, K, want_y=True,
+                                           want_boundary=True)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize(dev)
+    ts = []
+    for _ in range(max(args.steps, 1)):
+        dist.barrier(device_ids=[local])
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ts.append(e0.elapsed_time(e1))
+    ms = st_.median(ts)
+    (mx,) = max_over_ranks([ms], device=dev)
+    if rank == 0:
+        print(json.dumps({"metric": METRIC, "workload": "cp_prefill", "n_gpus": world, "steps": len(ts),
+                          "config": {"batch": w.batch, "context": w.L, "d_inner": w.D, "d_state": w.N, "block": K,
+                                     "io_dtype": w.io, "chunks": world},
+                          "ms": mx, "tokens_per_s": w.batch * w.L / (mx * 1e-3),
+                          "note": "chunk summary + one all-gather + carry fold + chunk prefill per rank"}),
+              flush=True)
+    dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -671,7 +741,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--workload", default="train",
-                    choices=["train", "train_fwd_bwd", "step65k", "step262k", "stack350m"],
+                    choices=["train", "train_fwd_bwd", "step65k", "step262k", "stack350m", "cp_prefill"],
                     help="train: the headline line; the others print their own measurement lines")
     args = ap.parse_args()
     if args.workload in ("step65k", "step262k"):
@@ -680,6 +750,8 @@ def main():
         return run_stack(args)
     if args.workload == "train_fwd_bwd":
         return run_train_step(args)
+    if args.workload == "cp_prefill":
+        return run_context_parallel(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

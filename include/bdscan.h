@@ -243,6 +243,33 @@ int bdscan_train_blocks_backward(const bdscan_dims *dims, const bdscan_inputs *i
                                  const float *boundary, const void *dy, const bdscan_grads *grads, void *ws,
                                  size_t ws_bytes, bdscan_stream_t stream);
 
+/* Context-parallel prefill, for a context split into consecutive chunks (for
+ * instance one per GPU, each chunk a whole number of blocks). The forward
+ * recurrence h_t = a_t h_{t-1} + b_t is affine in the state, so a chunk acts on
+ * its start state as h -> P h + H: P = the product of the chunk's decays a_t,
+ * H = the state the chunk reaches from zero. Composing the summaries of chunks
+ * 0 .. r-1 from h0 gives chunk r's start state; chunk r then runs
+ * bdscan_prefill from it. The pages describe the forward-only prefix operator
+ * whose block-end states are the cache (gist.science technical summary,
+ * "Methodik"); splitting its scan over chunks is this library's choice. */
+
+/* The chunk summary of in's whole context: H = forward state after the L
+ * tokens from a zero state, P = product over the L tokens of exp(delta A), both
+ * [batch, D, N] fp32 (written, required unless batch * D * N == 0). dims.block
+ * is not used beyond the argument checks. L == 0 gives H = 0, P = 1. One launch
+ * on `stream`, no scratch. */
+int bdscan_chunk_summary(const bdscan_dims *dims, const bdscan_inputs *in, float *H, float *P,
+                         bdscan_stream_t stream);
+
+/* h_in = the start state of chunk `index` of `chunks`: from h0 ([count] fp32,
+ * NULL = zero state), fold h = P_q * h + H_q for q = 0 .. index-1, where H_all
+ * and P_all hold the chunks' summaries one after another ([chunks][count] fp32,
+ * the layout of an all-gather of the per-chunk bdscan_chunk_summary outputs;
+ * may be NULL when index == 0); count = batch * D * N. h_in may not alias
+ * H_all or P_all. One launch on `stream`. */
+int bdscan_carry_fold(int64_t chunks, int64_t index, int64_t count, const float *h0, const float *H_all,
+                      const float *P_all, float *h_in, bdscan_stream_t stream);
+
 /* Human-readable name of a bdscan_status value (static storage). */
 const char *bdscan_status_string(int status);
 

@@ -53,11 +53,13 @@ _lib.bdscan_train_blocks_backward.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _v
                                               _vp]
 _lib.bdscan_train_blocks_backward_workspace.argtypes = [_P(Dims)]
 _lib.bdscan_train_blocks_backward_workspace.restype = ct.c_size_t
+_lib.bdscan_chunk_summary.argtypes = [_P(Dims), _P(Inputs), _vp, _vp, _vp]
+_lib.bdscan_carry_fold.argtypes = [ct.c_int64, ct.c_int64, ct.c_int64, _vp, _vp, _vp, _vp, _vp]
 _lib.bdscan_prefill_chunked_workspace.argtypes = [_P(Dims)]
 _lib.bdscan_prefill_chunked_workspace.restype = ct.c_size_t
 for _f in ("bdscan_train_blocks", "bdscan_prefill", "bdscan_block_step", "bdscan_commit_block",
            "bdscan_train_two_stream", "bdscan_full_bidirectional", "bdscan_prefill_chunked", "bdscan_prefill_chunked_noalloc",
-           "bdscan_train_blocks_backward", "bdscan_version"):
+           "bdscan_train_blocks_backward", "bdscan_chunk_summary", "bdscan_carry_fold", "bdscan_version"):
     getattr(_lib, _f).restype = ct.c_int
 _lib.bdscan_status_string.argtypes = [ct.c_int]
 _lib.bdscan_status_string.restype = ct.c_char_p
@@ -269,6 +271,38 @@ def train_blocks_backward(x, dt, A, B, C, Dskip, block, dy, boundary, z=None, h0
                                            ct.byref(gr), _ptr(ws), ws.numel() * ws.element_size(), _stream(dev))
     _check(rc, "bdscan_train_blocks_backward")
     return g
+
+
+def chunk_summary(x, dt, A, B, C, Dskip, block, dt_softplus=True, H=None, P=None):
+    """(H, P) of the context: the state it reaches from zero and the product of its decays, [batch, D, N]."""
+    dims, ins, (Bt, L, D, N), io, dev = _prepare(x, dt, A, B, C, Dskip, block, None, dt_softplus)
+    H = torch.empty((Bt, D, N), dtype=torch.float32, device=dev) if H is None else H
+    P = torch.empty((Bt, D, N), dtype=torch.float32, device=dev) if P is None else P
+    _need(H, "H", torch.float32, (Bt, D, N), dev)
+    _need(P, "P", torch.float32, (Bt, D, N), dev)
+    rc = _lib.bdscan_chunk_summary(ct.byref(dims), ct.byref(ins), _ptr(H), _ptr(P), _stream(dev))
+    _check(rc, "bdscan_chunk_summary")
+    return H, P
+
+
+def carry_fold(H_all, P_all, index, h0=None, out=None):
+    """Start state of chunk `index` from the chunks' summaries H_all, P_all ([chunks, batch, D, N]) and h0."""
+    if not isinstance(H_all, torch.Tensor) or H_all.dim() != 4:
+        raise ValueError("H_all must be a [chunks, batch, D, N] tensor")
+    _check_device(H_all.device)
+    dev = H_all.device
+    shape = tuple(H_all.shape)
+    _need(H_all, "H_all", torch.float32, shape, dev)
+    _need(P_all, "P_all", torch.float32, shape, dev)
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, shape[1:], dev)
+    out = torch.empty(shape[1:], dtype=torch.float32, device=dev) if out is None else out
+    _need(out, "out", torch.float32, shape[1:], dev)
+    count = shape[1] * shape[2] * shape[3]
+    rc = _lib.bdscan_carry_fold(shape[0], int(index), count, _ptr(h0), _ptr(H_all), _ptr(P_all), _ptr(out),
+                                _stream(dev))
+    _check(rc, "bdscan_carry_fold")
+    return out
 
 
 def block_step(x, dt, A, B, C, Dskip, h_cache, z=None, dt_softplus=True, y=None):

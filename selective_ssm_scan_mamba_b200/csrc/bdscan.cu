@@ -255,6 +255,34 @@ int launch_bwd(const bdk::BwdArgs &a, int64_t batch, int64_t ct, void *dB, void 
     return BDSCAN_OK;
 }
 
+// ---- context-parallel pieces: the fold of gathered chunk summaries ------------
+// h_in = P_{r-1} (... (P_0 h0 + H_0) ...) + H_{r-1}: the forward state at the
+// start of chunk r, from the (H, P) summaries of chunks 0 .. r-1 ([chunks][count]).
+__global__ void __launch_bounds__(256) bdscan_carry_fold_kernel(const float *__restrict__ h0,
+                                                                const float *__restrict__ H,
+                                                                const float *__restrict__ P, int64_t count,
+                                                                int64_t upto, float *__restrict__ h_in) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
+        float h = h0 ? h0[i] : 0.f;
+        for (int64_t q = 0; q < upto; ++q) h = __fmaf_rn(P[q * count + i], h, H[q * count + i]);
+        h_in[i] = h;
+    }
+}
+
+// the summary of an empty context: H = 0, P = 1
+__global__ void __launch_bounds__(256) bdscan_identity_summary_kernel(float *H, float *P, int64_t count) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
+        H[i] = 0.f;
+        P[i] = 1.f;
+    }
+}
+
+unsigned elementwise_blocks(int64_t count) {
+    int64_t blocks = (count + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    return (unsigned)(blocks > 0 ? blocks : 1);
+}
+
 // ---- allocation-free variant of the time-chunked prefill -----------------------
 // Scratch for bdscan_prefill_chunked_noalloc: a fixed array in device global
 // memory, created when the library is loaded on a device and kept until the
@@ -372,6 +400,42 @@ int bdscan_train_blocks_backward(const bdscan_dims *dims, const bdscan_inputs *i
                                  : launch_bwd<__nv_bfloat16, 64>(a, dm->batch, p.ct, gr->dB, gr->dC, gr->dA, gr->dDskip, st);
     return dm->d_state == 16 ? launch_bwd<float, 16>(a, dm->batch, p.ct, gr->dB, gr->dC, gr->dA, gr->dDskip, st)
                              : launch_bwd<float, 64>(a, dm->batch, p.ct, gr->dB, gr->dC, gr->dA, gr->dDskip, st);
+}
+
+int bdscan_chunk_summary(const bdscan_dims *dims, const bdscan_inputs *in, float *H, float *P,
+                         bdscan_stream_t stream) {
+    int rc = check_common(dims, in);
+    if (rc != BDSCAN_OK) return rc;
+    const int64_t count = dims->batch * dims->d_inner * dims->d_state;
+    if (count == 0) return BDSCAN_OK;
+    if (!H || !P) return BDSCAN_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dims->seqlen == 0) {
+        bdscan_identity_summary_kernel<<<elementwise_blocks(count), 256, 0, st>>>(H, P, count);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
+        return BDSCAN_OK;
+    }
+    // the first pass of the time-chunked prefill, over one chunk: the whole context
+    Chunking c;
+    c.len = dims->seqlen;
+    c.count = 1;
+    c.pass = 1;
+    c.ws_h = H;
+    c.ws_p = P;
+    return run(kCleanStream, dims, in, nullptr, nullptr, nullptr, nullptr, stream, nullptr, &c);
+}
+
+int bdscan_carry_fold(int64_t chunks, int64_t index, int64_t count, const float *h0, const float *H_all,
+                      const float *P_all, float *h_in, bdscan_stream_t stream) {
+    if (chunks < 1 || index < 0 || index >= chunks || count < 0) return BDSCAN_ERR_INVALID_ARG;
+    if (count == 0) return BDSCAN_OK;
+    if (!h_in || (index > 0 && (!H_all || !P_all))) return BDSCAN_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    bdscan_carry_fold_kernel<<<elementwise_blocks(count), 256, 0, st>>>(h0, H_all, P_all, count, index, h_in);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
+    return BDSCAN_OK;
 }
 
 int bdscan_train_blocks(const bdscan_dims *dims, const bdscan_inputs *in, const float *h0, void *y,
