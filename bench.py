@@ -41,11 +41,16 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "train_traffic.json")
 
 
 def kernel_source_hash() -> str:
-    """Hash of the sources the forward scan kernel is compiled from (its
-    device code; host-side launch code and other kernels do not change it)."""
+    """Hash of the code the forward scan kernel is compiled from (its device
+    sources, with comments and whitespace removed: host-side launch code,
+    other kernels and comment edits do not change it)."""
+    import re
     h = hashlib.sha256()
     for name in ("bdscan_device.cuh", "bdscan_kernels.cuh"):
-        h.update(open(os.path.join(ROOT, "selective_ssm_scan_mamba_b200", "csrc", name), "rb").read())
+        src = open(os.path.join(ROOT, "selective_ssm_scan_mamba_b200", "csrc", name)).read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update("".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -98,10 +98,11 @@ struct Cfg {
     static constexpr int SPAN = MODE == kFused ? (KC > 0 ? KC : T) : 16;
     static constexpr bool KEEP_B = SPAN <= 16 && N == 16;                        // keep b for phase C
     static constexpr int PER = T / W > 0 ? T / W : 1;                            // readout tokens per warp
-    // whole-block fused variants keep a block's decays and inputs in TMEM (8
-    // columns per token: a[4], b[4]). Warp w uses lane quadrant w % 4 and
-    // column range (w / 4) * WCOLS; a CTA's columns fit the SM's 512 even at
-    // the largest residency these variants reach (N = 16, K = 32: 2 CTAs x 256).
+    // whole-block fused variants (and the long fused mode, span by span) keep a
+    // span's decays and inputs in TMEM (8 columns per token: a[4], b[4]). Warp
+    // w uses lane quadrant w % 4 and column range (w / 4) * WCOLS; a CTA's
+    // columns fit the SM's 512 at the residency each variant reaches (N = 16:
+    // 3 CTAs x 128 for spans of 16, 2 CTAs x 256 for K = 32; N = 64: 1 x 512).
     static constexpr int WCOLS = SPAN * 2 * NPT;
     static constexpr int TNEED = (W / 4) * WCOLS;
     static constexpr bool TMEM = ((MODE == kFused && KC > 0) || MODE == kLongFused) && W % 4 == 0 && NPT == 4 &&
