@@ -54,13 +54,13 @@ bool long_fused_fits(int64_t K) {
     return bdk::Layout<IO, N, bdk::kLongFused, 0>::base_bytes + long_fused_ck_bytes(K, N) <= (size_t)kMaxDynSmem;
 }
 
-template <class IO, int N, int MODE, int KC>
+template <class IO, int N, int MODE, int KC, int NPTV = 4>
 int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1) {
-    using CF = bdk::Cfg<N, MODE, KC>;
-    using LY = bdk::Layout<IO, N, MODE, KC>;
+    using CF = bdk::Cfg<N, MODE, KC, NPTV>;
+    using LY = bdk::Layout<IO, N, MODE, KC, NPTV>;
     const size_t smem = LY::base_bytes + (MODE == bdk::kLong ? (size_t)a.K * bdk::kCh * 4
                                           : MODE == bdk::kLongFused ? long_fused_ck_bytes(a.K, N) : 0);
-    auto kern = bdk::bdscan_kernel<IO, N, MODE, KC>;
+    auto kern = bdk::bdscan_kernel<IO, N, MODE, KC, NPTV>;
     // raise the dynamic shared-memory ceiling once per device
     static std::atomic<uint64_t> done_mask{0};
     int dev = 0;
@@ -81,7 +81,18 @@ int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz =
 }
 
 template <class IO, int N>
-int dispatch_mode(int mode, const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1) {
+int dispatch_mode(int mode, const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1,
+                  bool thin = false) {
+    if constexpr (N == 16) {
+        if (thin && mode == bdk::kFused) {   // one state per lane: the latency-bound small block step
+            switch (a.K) {
+                case 4: return launch<IO, N, bdk::kFused, 4, 1>(a, batch, st);
+                case 16: return launch<IO, N, bdk::kFused, 16, 1>(a, batch, st);
+                case 32: return launch<IO, N, bdk::kFused, 32, 1>(a, batch, st);
+                default: return launch<IO, N, bdk::kFused, 0, 1>(a, batch, st);
+            }
+        }
+    }
     if (mode == bdk::kForwardOnly) return launch<IO, N, bdk::kForwardOnly, 0>(a, batch, st, gz);
     if (mode == bdk::kLong) return launch<IO, N, bdk::kLong, 0>(a, batch, st);
     if (mode == bdk::kLongFused) return launch<IO, N, bdk::kLongFused, 0>(a, batch, st);
@@ -147,10 +158,17 @@ int run(Op op, const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, 
     const unsigned gz = ch ? (unsigned)ch->count : 1u;
     a.L = dm->seqlen; a.D = dm->d_inner; a.K = (int32_t)dm->block; a.dt_softplus = dm->dt_softplus;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // a block step (or a commit with y) over at most one CTA per SM runs thin
+    bool thin = false;
+    if ((op == kStep || (op == kCommit && y)) && mode == bdk::kFused && dm->d_state == 16) {
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        thin = dm->batch * ((dm->d_inner + bdk::kCh - 1) / bdk::kCh) <= sms;
+    }
     if (dm->io_dtype == BDSCAN_BF16)
-        return dm->d_state == 16 ? dispatch_mode<__nv_bfloat16, 16>(mode, a, dm->batch, st, gz)
+        return dm->d_state == 16 ? dispatch_mode<__nv_bfloat16, 16>(mode, a, dm->batch, st, gz, thin)
                                  : dispatch_mode<__nv_bfloat16, 64>(mode, a, dm->batch, st, gz);
-    return dm->d_state == 16 ? dispatch_mode<float, 16>(mode, a, dm->batch, st, gz)
+    return dm->d_state == 16 ? dispatch_mode<float, 16>(mode, a, dm->batch, st, gz, thin)
                              : dispatch_mode<float, 64>(mode, a, dm->batch, st, gz);
 }
 

@@ -79,17 +79,15 @@ struct ScanArgs {
     int32_t K, dt_softplus;
 };
 
-// States per lane: 4 in every mode (one warp per 4 states). Prefills of too
-// few channels to fill the GPU get their parallelism from time chunks
-// (bdscan_prefill_chunked), not from thinner lanes.
-template <int N, int MODE>
-struct Npt {
-    static constexpr int value = 4;
-};
-
-template <int N, int MODE, int KC>
+// NPTV = states per lane: 4 (one warp per 4 states) everywhere but the thin
+// block-step variant, 1 state per lane (16 warps per CTA at N = 16), which a
+// block step of too few channels to fill the GPU uses: its 32 tokens are a
+// latency chain, and a quarter of the per-token work per warp shortens it.
+// Prefills of too few channels get their parallelism from time chunks
+// (bdscan_prefill_chunked) instead.
+template <int N, int MODE, int KC, int NPTV = 4>
 struct Cfg {
-    static constexpr int NPT = Npt<N, MODE>::value;
+    static constexpr int NPT = NPTV;
     static constexpr int W = N / NPT;                 // warps per CTA (state groups)
     static constexpr int THREADS = 32 * W;
     static constexpr int T = (MODE == kFused && (KC == 0 || KC > 16 || (KC == 16 && N == 16))) ? 32
@@ -116,9 +114,9 @@ struct Cfg {
 };
 
 // Shared-memory carve-up (bytes; every offset is a multiple of 16).
-template <class IO, int N, int MODE, int KC>
+template <class IO, int N, int MODE, int KC, int NPTV = 4>
 struct Layout {
-    using CF = Cfg<N, MODE, KC>;
+    using CF = Cfg<N, MODE, KC, NPTV>;
     static constexpr int T = CF::T, S = CF::S, W = CF::W;
     static constexpr int RP = T + 4;                       // padded row of the readout buffer
     static constexpr int xb = T * kCh * (int)sizeof(IO);   // one x / dt / z tile
@@ -236,11 +234,11 @@ __device__ __forceinline__ void stage_tile(char *st, const ScanArgs &a, int64_t 
 // One CTA = one (batch row, 32-channel tile). MODE selects forward-only, fused
 // (block <= 32; KC = compile-time block length, or 0 for a runtime one), or
 // the long-block two-sweep path.
-template <class IO, int N, int MODE, int KC>
-__global__ void __launch_bounds__(Cfg<N, MODE, KC>::THREADS, Cfg<N, MODE, KC>::MINB)
+template <class IO, int N, int MODE, int KC, int NPTV = 4>
+__global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, KC, NPTV>::MINB)
     bdscan_kernel(const ScanArgs a) {
-    using CF = Cfg<N, MODE, KC>;
-    using LY = Layout<IO, N, MODE, KC>;
+    using CF = Cfg<N, MODE, KC, NPTV>;
+    using LY = Layout<IO, N, MODE, KC, NPTV>;
     constexpr int NPT = CF::NPT, W = CF::W, NT = CF::THREADS, T = CF::T, S = CF::S, SPAN = CF::SPAN;
     constexpr int RP = LY::RP, PER = CF::PER;
     constexpr bool KEEP_B = CF::KEEP_B;
