@@ -51,11 +51,6 @@ def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     return r.astype(np.uint16)
 
 
-def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
-    """Exact widening of bf16 bit patterns to fp32."""
-    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
-
-
 def _rng(seed: int, *key: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence([int(seed), *map(int, key)])))
 
