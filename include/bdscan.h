@@ -69,7 +69,7 @@ typedef enum {
     BDSCAN_OK = 0,
     BDSCAN_ERR_INVALID_ARG = 1,  /* NULL required pointer, negative size, L % K != 0, ... */
     BDSCAN_ERR_UNSUPPORTED = 2,  /* N not 16/64, D not a multiple of the vector width,
-                                    K > 768 for a pass with a reverse scan */
+                                    a block too long for a pass with a reverse scan */
     BDSCAN_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned */
     BDSCAN_ERR_WORKSPACE = 4,    /* workspace missing or smaller than the size the library asks for */
     BDSCAN_ERR_CUDA = 5          /* a kernel launch failed; see bdscan_last_cuda_error() */
@@ -102,8 +102,12 @@ typedef struct {
  * block-confined reverse scan of each block; y = (y_fwd + y_rev) * gate.
  * Optional outputs: boundary states after each block (NULL = not written) and
  * the final state h_out (NULL = not written). Blocks longer than 32 tokens
- * take a two-sweep path that stages the block's reverse readout in shared
- * memory, which limits K to 768; longer blocks return BDSCAN_ERR_UNSUPPORTED.
+ * first sweep the reverse state alone and keep its value at every 16-token
+ * span start in shared memory ((ceil(K/16) - 1) x N x 128 bytes: K up to 1392
+ * at N = 16 and 304 at N = 64 with bf16 I/O, 1200 and 240 with fp32), then run
+ * the fused pass span by span. Where that does not fit, a two-sweep path stages
+ * the block's reverse readout in shared memory instead (K <= 768); blocks too
+ * long for both return BDSCAN_ERR_UNSUPPORTED.
  * Source: full-block objective, gist.science technical summary, "Methodik";
  * cache agreement, "Wesentliche Beitraege". */
 int bdscan_train_blocks(const bdscan_dims *dims, const bdscan_inputs *in,
