@@ -170,6 +170,17 @@ def _oracle_worker(conn, name, seed, n_seq, c0, c1):
         conn.send("done")
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (first processor in /proc/cpuinfo), or ''."""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return ""
+
+
 class OraclePool:
     """The fp64 oracle, unchanged, on every host core: `workers` spawned
     processes each own a contiguous slice of the channels (channels are
@@ -234,7 +245,7 @@ def run_reference(args):
         "config": {"workload": WORKLOAD, "batch": w.batch, "seq_len": w.L, "d_inner": w.D, "d_state": w.N,
                    "block": w.K, "io_dtype": w.io, "parallelism": f"dp{args.gpus}", "sample": sample},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": pool.workers, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu": cpu_model()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -387,7 +398,7 @@ def run_ours(args):
             pool.close()
         cpu = {"value": pool.tokens_per_step() / secs, "unit": "tokens/s", "cores": pool.workers, "kind": "oracle",
                "sample": f"all {w.batch} sequences x {w.L} tokens x {w.D} channels once, channels split over "
-                         f"{pool.workers} processes, {secs:.1f} s"}
+                         f"{pool.workers} processes, {secs:.1f} s", "cpu": cpu_model()}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -401,6 +412,7 @@ def run_ours(args):
                      "peak_source": f"16 MUFU.EX2/clk/SM x {SM_COUNT} SMs x {peaks['sm_max_mhz']:.0f} MHz",
                      "hbm": {"achieved": hbm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                              "frac": hbm_gbs / peaks["hbm_gbs"], "peak_source": peaks["source"],
+                             "frac_of_nominal_8000": hbm_gbs / 8000.0,
                              "algorithmic_bytes_per_launch": nbytes},
                      "kernel_ms": launch_ms},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
