@@ -109,3 +109,67 @@ def test_status_strings(lib):
     assert lib.bdscan_status_string(3) == b"BDSCAN_ERR_ALIGNMENT"
     assert lib.bdscan_status_string(99) == b"BDSCAN_UNKNOWN_STATUS"
     assert lib.bdscan_version() >= 100
+
+
+class Grads(C.Structure):
+    _fields_ = [("dx", C.c_void_p), ("ddt", C.c_void_p), ("dz", C.c_void_p), ("dB", C.c_void_p),
+                ("dC", C.c_void_p), ("dA", C.c_void_p), ("dDskip", C.c_void_p), ("dh0", C.c_void_p)]
+
+
+def _grads(**kw):
+    d = dict(dx=P + 0x1000, ddt=P + 0x1100, dz=None, dB=P + 0x1200, dC=P + 0x1300, dA=P + 0x1400,
+             dDskip=P + 0x1500, dh0=None)
+    d.update(kw)
+    return Grads(**d)
+
+
+def _ws_floats(Bt, L, D, N, K):
+    r4 = lambda v: (v + 3) // 4 * 4  # noqa: E731
+    ct = (D + 31) // 32
+    ntb = (K + 7) // 8 if K > 8 else 1
+    nck = ntb - 2 if ntb > 2 else 0
+    return r4(Bt * ct * L * 2 * N) + r4(Bt * D * N) + r4(Bt * D) + Bt * ct * nck * (N // 4) * 32 * 8
+
+
+@pytest.mark.parametrize("Bt,L,D,N,K", [(8, 4096, 1536, 16, 16), (2, 96, 72, 16, 3), (1, 256, 40, 64, 64),
+                                        (3, 0, 64, 16, 16), (1, 768, 24, 16, 256)])
+def test_backward_workspace_size(lib, Bt, L, D, N, K):
+    lib.bdscan_train_blocks_backward_workspace.argtypes = [C.POINTER(Dims)]
+    lib.bdscan_train_blocks_backward_workspace.restype = C.c_size_t
+    d = Dims(Bt, L, D, N, K, 1, 1)
+    assert lib.bdscan_train_blocks_backward_workspace(C.byref(d)) == 4 * _ws_floats(Bt, L, D, N, K)
+    assert lib.bdscan_train_blocks_backward_workspace(C.byref(Dims(Bt, L, D, 32, K, 1, 1))) == 0
+
+
+@pytest.mark.parametrize("ins,grads,bnd,dy,ws_bytes,want", [
+    (_ins(), _grads(dx=None), P + 0x2000, P + 0x2100, 1 << 30, 1),           # dx missing
+    (_ins(), _grads(dB=None), P + 0x2000, P + 0x2100, 1 << 30, 1),           # dB missing
+    (_ins(), _grads(dA=None), P + 0x2000, P + 0x2100, 1 << 30, 1),           # dA missing
+    (_ins(), _grads(), P + 0x2000, None, 1 << 30, 1),                        # dy missing
+    (_ins(), _grads(), None, P + 0x2100, 1 << 30, 1),                        # boundary states needed for L > K
+    (_ins(z=P + 0x600), _grads(), P + 0x2000, P + 0x2100, 1 << 30, 1),      # z given, dz missing
+    (_ins(), _grads(), P + 0x2000, P + 0x2104, 1 << 30, 3),                  # dy misaligned
+    (_ins(), _grads(), P + 0x2000, P + 0x2100, 1024, 4),                     # workspace too small
+])
+def test_backward_rejects(lib, ins, grads, bnd, dy, ws_bytes, want):
+    lib.bdscan_train_blocks_backward.argtypes = [C.POINTER(Dims), C.POINTER(Inputs), C.c_void_p, C.c_void_p,
+                                                 C.c_void_p, C.POINTER(Grads), C.c_void_p, C.c_size_t, C.c_void_p]
+    d = Dims(2, 64, 64, 16, 16, 1, 1)
+    assert lib.bdscan_train_blocks_backward(C.byref(d), C.byref(ins), None, bnd, dy, C.byref(grads), P + 0x4000,
+                                            ws_bytes, None) == want
+
+
+def test_context_parallel_pieces_reject(lib):
+    lib.bdscan_carry_fold.argtypes = [C.c_int64, C.c_int64, C.c_int64] + [C.c_void_p] * 5
+    lib.bdscan_chunk_summary.argtypes = [C.POINTER(Dims), C.POINTER(Inputs)] + [C.c_void_p] * 3
+    fold = lib.bdscan_carry_fold
+    assert fold(0, 0, 16, None, None, None, P, None) == 1          # no chunks
+    assert fold(2, 2, 16, None, None, None, P, None) == 1          # index out of range
+    assert fold(2, -1, 16, None, None, None, P, None) == 1
+    assert fold(2, 1, -4, None, None, None, P, None) == 1          # negative count
+    assert fold(2, 1, 16, None, None, None, P, None) == 1          # summaries needed past chunk 0
+    assert fold(2, 1, 16, None, P, P, None, None) == 1             # no output
+    assert fold(2, 1, 0, None, None, None, None, None) == 0        # nothing to do
+    d = Dims(2, 64, 64, 16, 16, 1, 1)
+    assert lib.bdscan_chunk_summary(C.byref(d), C.byref(_ins()), None, P, None) == 1
+    assert lib.bdscan_chunk_summary(C.byref(Dims(2, 64, 64, 32, 16, 1, 1)), C.byref(_ins()), P, P, None) == 2
