@@ -367,9 +367,48 @@ def check_backward_homogeneity(mutant=0):
     return True, ""
 
 
+def check_backward_single_token_closed_form(mutant=0):
+    """One token (L = K = 1): with a = exp(delta A), the pre-gate output is
+    s = sum_n C_n (a_n h0_n + 2 delta x B_n) + 2 Dskip x, y = s silu(z), and
+    every gradient has a closed form written out here from that expression:
+    ds/dx = sum_n 2 delta B_n C_n + 2 Dskip, ds/dB_n = 2 delta x C_n,
+    ds/dC_n = a_n h0_n + 2 delta x B_n, ds/dh0_n = C_n a_n,
+    ds/ddelta = sum_n C_n (A_n a_n h0_n + 2 x B_n), ds/dA_n = C_n delta a_n h0_n,
+    ds/dDskip = 2 x; dy/ds = silu(z), dy/dz = s sigmoid(z) (1 + z (1 - sigmoid(z)))."""
+    Bt, D, N = 2, 3, 4
+    v = _bwd_case(600, Bt, 1, D, N, True, True, True)
+    g = oracle.train_blocks_backward(v["x"], v["dt"], v["A"], v["B"], v["C"], v["Dskip"], 1, v["dy"], z=v["z"],
+                                     h0=v["h0"], dt_softplus=True, mutant=mutant)
+    x, dt, z, dy = v["x"][:, 0], v["dt"][:, 0], v["z"][:, 0], v["dy"][:, 0]          # [Bt, D]
+    B, C = v["B"][:, 0], v["C"][:, 0]                                                # [Bt, N]
+    A, Dk, h0 = v["A"], v["Dskip"], v["h0"]                                          # [D, N], [D], [Bt, D, N]
+    dl = np.log1p(np.exp(dt))                                                        # softplus
+    a = np.exp(dl[:, :, None] * A[None])                                             # [Bt, D, N]
+    s = np.einsum("bn,bdn->bd", C, a * h0) + 2 * dl * x * np.einsum("bn,bn->b", B, C)[:, None] + 2 * Dk * x
+    sg = 1 / (1 + np.exp(-z))
+    ds = dy * z * sg
+    want = {
+        "dx": ds * (2 * dl * np.einsum("bn,bn->b", B, C)[:, None] + 2 * Dk),
+        "ddt": ds * (np.einsum("bn,bdn->bd", C, A[None] * a * h0) + 2 * x * np.einsum("bn,bn->b", B, C)[:, None])
+               * (1 / (1 + np.exp(-dt))),
+        "dz": dy * s * sg * (1 + z * (1 - sg)),
+        "dB": 2 * np.einsum("bd,bn->bn", ds * dl * x, C),
+        "dC": np.einsum("bd,bdn->bn", ds, a * h0) + 2 * np.einsum("bd,bn->bn", ds * dl * x, B),
+        "dA": np.einsum("bd,bn,bdn->dn", ds * dl, C, a * h0),
+        "dDskip": np.sum(2 * x * ds, axis=0),
+        "dh0": ds[:, :, None] * C[:, None, :] * a,
+    }
+    for k, w in want.items():
+        got = g[k][:, 0] if k in ("dx", "ddt", "dz", "dB", "dC") else g[k]
+        if not _close(got, w, rtol=1e-12, atol=1e-13):
+            return False, f"{k}: {np.max(np.abs(got - w))}"
+    return True, ""
+
+
 ALL_CHECKS = [
     check_hand_example, check_softplus_closed_forms, check_block1_closed_form, check_blockL_flip,
     check_bruteforce, check_steady_state, check_linearity, check_zero_limits, check_commit_chain,
     check_prefix_only, check_block_locality, check_two_stream,
     check_backward_finite_differences, check_backward_linear_in_x, check_backward_homogeneity,
+    check_backward_single_token_closed_form,
 ]
