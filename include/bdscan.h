@@ -155,7 +155,10 @@ int bdscan_prefill_chunked(const bdscan_dims *dims, const bdscan_inputs *in, con
  * BDSCAN_ERR_WORKSPACE (use bdscan_prefill_chunked with your own buffer).
  * The first call on a device looks up the array's device address (a CUDA
  * runtime query, done once per device); make that first call before any
- * stream capture. All calls share the one array and it keeps whatever the
+ * stream capture. The address is kept for the life of the process, so the
+ * entry point must not be used on a device after cudaDeviceReset, nor from a
+ * context other than the device's primary context (the runtime's default):
+ * the library's device memory then sits at another address. All calls share the one array and it keeps whatever the
  * last call left there; nothing in it has to start at zero, because each
  * call's first pass writes every entry its second pass reads. Calls that may
  * run at the same time on the GPU (different streams with no ordering between

@@ -111,8 +111,24 @@ struct Chunking {   // time-chunked prefill: chunk length, chunk count, pass, wo
     float *ws_h = nullptr, *ws_p = nullptr;
 };
 
-int run(Op op, const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, void *y, float *h_out,
-        float *boundary, bdscan_stream_t stream, const float *blk_h0 = nullptr, const Chunking *ch = nullptr) {
+// Number of SMs of the current device, queried once per device.
+int device_sm_count() {
+    static std::atomic<int> sms[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    int n = sms[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        sms[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
+// Every argument check of one pass, and the kernel mode it selects; queues
+// nothing. Multi-pass entry points call this for all their passes before the
+// first launch, so a call that returns an error has queued no work.
+int validate(Op op, const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, const void *y,
+             const float *h_out, const float *boundary, int *mode_out) {
     int rc = check_common(dm, in);
     if (rc != BDSCAN_OK) return rc;
     if ((op == kStep || op == kCommit) && dm->seqlen != dm->block) return BDSCAN_ERR_INVALID_ARG;
@@ -145,6 +161,15 @@ int run(Op op, const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, 
             mode = bdk::kLong;
         }
     }
+    if (mode_out) *mode_out = mode;
+    return BDSCAN_OK;
+}
+
+int run(Op op, const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, void *y, float *h_out,
+        float *boundary, bdscan_stream_t stream, const float *blk_h0 = nullptr, const Chunking *ch = nullptr) {
+    int mode = 0;
+    const int rc = validate(op, dm, in, h0, y, h_out, boundary, &mode);
+    if (rc != BDSCAN_OK) return rc;
     if (dm->batch == 0 || dm->d_inner == 0) return BDSCAN_OK;   // nothing to compute or write
 
     bdk::ScanArgs a;
@@ -160,11 +185,8 @@ int run(Op op, const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // a block step (or a commit with y) over at most one CTA per SM runs thin
     bool thin = false;
-    if ((op == kStep || (op == kCommit && y)) && mode == bdk::kFused && dm->d_state == 16) {
-        int dev = 0, sms = 148;
-        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        thin = dm->batch * ((dm->d_inner + bdk::kCh - 1) / bdk::kCh) <= sms;
-    }
+    if ((op == kStep || (op == kCommit && y)) && mode == bdk::kFused && dm->d_state == 16)
+        thin = dm->batch * ((dm->d_inner + bdk::kCh - 1) / bdk::kCh) <= device_sm_count();
     if (dm->io_dtype == BDSCAN_BF16)
         return dm->d_state == 16 ? dispatch_mode<__nv_bfloat16, 16>(mode, a, dm->batch, st, gz, thin)
                                  : dispatch_mode<__nv_bfloat16, 64>(mode, a, dm->batch, st, gz);
@@ -179,8 +201,7 @@ int run(Op op, const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, 
 // length is a multiple of 16 tokens.
 Chunking chunk_plan(const bdscan_dims *dm) {
     Chunking c;
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = device_sm_count();
     const int64_t row_ctas = dm->batch * ((dm->d_inner + bdk::kCh - 1) / bdk::kCh);
     int64_t g = (row_ctas > 0 && row_ctas < sms) ? (3 * (int64_t)sms + row_ctas - 1) / row_ctas : 1;
     const int64_t gmax_len = dm->seqlen / 256 > 0 ? dm->seqlen / 256 : 1;
@@ -201,6 +222,13 @@ size_t chunked_ws_bytes(const bdscan_dims *dm, const Chunking &c) {
     return 2 * (size_t)dm->batch * (size_t)c.count * (size_t)dm->d_inner * (size_t)dm->d_state * sizeof(float);
 }
 
+// Argument checks of both passes of the time-chunked prefill (queues nothing).
+int check_chunked_passes(const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, const void *y,
+                         const float *h_out, const float *boundary) {
+    const int rc = validate(kCleanStream, dm, in, nullptr, nullptr, nullptr, nullptr, nullptr);
+    return rc != BDSCAN_OK ? rc : validate(kPrefill, dm, in, h0, y, h_out, boundary, nullptr);
+}
+
 // The two passes of the time-chunked prefill on caller-provided scratch
 // (ws: 2 * batch * chunks * D * N floats, 16-byte aligned).
 int prefill_chunked_on(const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, void *y, float *h_out,
@@ -208,11 +236,14 @@ int prefill_chunked_on(const bdscan_dims *dm, const bdscan_inputs *in, const flo
     Chunking c = chunk_plan(dm);
     if (c.count <= 1)   // enough parallelism without chunks: the sequential scan (bit-identical caches)
         return run(kPrefill, dm, in, h0, y, h_out, boundary, stream);
+    // both passes' checks before the first launch (pass 2 alone needs h_out, y, boundary)
+    int rc = check_chunked_passes(dm, in, h0, y, h_out, boundary);
+    if (rc != BDSCAN_OK) return rc;
     const size_t half = (size_t)dm->batch * c.count * dm->d_inner * dm->d_state;
     c.ws_h = ws;
     c.ws_p = ws + half;
     c.pass = 1;
-    int rc = run(kCleanStream, dm, in, nullptr, nullptr, nullptr, nullptr, stream, nullptr, &c);
+    rc = run(kCleanStream, dm, in, nullptr, nullptr, nullptr, nullptr, stream, nullptr, &c);
     if (rc != BDSCAN_OK) return rc;
     c.pass = 2;
     return run(kPrefill, dm, in, h0, y, h_out, boundary, stream, nullptr, &c);
@@ -340,7 +371,7 @@ extern "C" {
 
 int bdscan_prefill_chunked_noalloc(const bdscan_dims *dims, const bdscan_inputs *in, const float *h0, void *y,
                                    float *h_out, float *boundary, bdscan_stream_t stream) {
-    int rc = check_common(dims, in);
+    int rc = check_chunked_passes(dims, in, h0, y, h_out, boundary);
     if (rc != BDSCAN_OK) return rc;
     const size_t need = chunked_ws_bytes(dims, chunk_plan(dims));
     if (need > kStaticScratchFloats * sizeof(float)) return BDSCAN_ERR_WORKSPACE;   // beyond the fixed scratch
@@ -485,6 +516,10 @@ int bdscan_train_two_stream(const bdscan_dims *dims, const bdscan_inputs *clean,
     if (rc != BDSCAN_OK) return rc;
     const bool any_block = dims->batch * dims->d_inner > 0 && dims->seqlen > 0;
     if (any_block && !boundary) return BDSCAN_ERR_INVALID_ARG;
+    // both passes' checks (y_noisy, the long-block mode) before the first launch
+    rc = validate(kCleanStream, dims, clean, h0, y_clean, h_out, boundary, nullptr);
+    if (rc == BDSCAN_OK) rc = validate(kTrain, dims, noisy, h0, y_noisy, nullptr, nullptr, nullptr);
+    if (rc != BDSCAN_OK) return rc;
     // the clean stream: forward-only scan writing the block caches (and y_clean)
     rc = run(kCleanStream, dims, clean, h0, y_clean, h_out, boundary, stream);
     if (rc != BDSCAN_OK) return rc;
@@ -497,10 +532,13 @@ int bdscan_full_bidirectional(const bdscan_dims *dims, const bdscan_inputs *in, 
     if (!dims || !in) return BDSCAN_ERR_INVALID_ARG;
     bdscan_inputs ungated = *in;
     ungated.z = nullptr;
-    // forward pass: y = y_fwd + Dskip x (ungated)
-    int rc = run(kCleanStream, dims, &ungated, h0, y, h_out, nullptr, stream);
+    // both passes' checks (y is required by the second) before the first launch
+    int rc = validate(kCleanStream, dims, &ungated, h0, y, h_out, nullptr, nullptr);
+    if (rc == BDSCAN_OK) rc = validate(kReverseAccumulate, dims, in, nullptr, y, nullptr, nullptr, nullptr);
     if (rc != BDSCAN_OK) return rc;
-    if (dims->batch * dims->seqlen * dims->d_inner > 0 && !y) return BDSCAN_ERR_INVALID_ARG;
+    // forward pass: y = y_fwd + Dskip x (ungated)
+    rc = run(kCleanStream, dims, &ungated, h0, y, h_out, nullptr, stream);
+    if (rc != BDSCAN_OK) return rc;
     // reverse pass over the whole sequence: y = (y + y_rev + Dskip x) * gate
     return run(kReverseAccumulate, dims, in, nullptr, y, nullptr, nullptr, stream);
 }

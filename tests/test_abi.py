@@ -173,3 +173,67 @@ def test_context_parallel_pieces_reject(lib):
     d = Dims(2, 64, 64, 16, 16, 1, 1)
     assert lib.bdscan_chunk_summary(C.byref(d), C.byref(_ins()), None, P, None) == 1
     assert lib.bdscan_chunk_summary(C.byref(Dims(2, 64, 64, 32, 16, 1, 1)), C.byref(_ins()), P, P, None) == 2
+
+
+# Multi-pass entry points: the second pass's checks (a missing or misaligned
+# output, a block too long for any reverse-scan mode) must reject the call
+# before the first pass is queued. The pointers are fake; on this CPU-only
+# check a launch would surface as BDSCAN_ERR_CUDA (5), so getting the argument
+# error instead shows that nothing was launched. Never run with a device
+# visible: fake pointers must not reach a GPU.
+def _no_device():
+    try:
+        import torch
+        return not torch.cuda.is_available()
+    except Exception:
+        return True
+
+
+cpu_only = pytest.mark.skipif(not _no_device(), reason="fake device pointers: CPU-only check")
+
+
+@cpu_only
+def test_full_bidirectional_checks_both_passes_first(lib):
+    lib.bdscan_full_bidirectional.argtypes = [C.POINTER(Dims), C.POINTER(Inputs)] + [C.c_void_p] * 4
+    d = Dims(2, 64, 64, 16, 64, 1, 1)
+    f = lib.bdscan_full_bidirectional
+    assert f(C.byref(d), C.byref(_ins()), None, None, P + 0x700, None) == 1            # y required
+    assert f(C.byref(d), C.byref(_ins()), None, P + 0x604, P + 0x700, None) == 3       # y misaligned
+    assert f(C.byref(d), C.byref(_ins(z=P + 0x608)), None, P + 0x600, None, None) == 3  # gate misaligned
+
+
+@cpu_only
+def test_train_two_stream_checks_both_passes_first(lib):
+    lib.bdscan_train_two_stream.argtypes = [C.POINTER(Dims), C.POINTER(Inputs), C.POINTER(Inputs)] + \
+        [C.c_void_p] * 6
+    f = lib.bdscan_train_two_stream
+    d = Dims(2, 64, 64, 16, 16, 1, 1)
+    # y_noisy missing
+    assert f(C.byref(d), C.byref(_ins()), C.byref(_ins()), None, None, None, P + 0x800, None, None) == 1
+    # y_noisy misaligned
+    assert f(C.byref(d), C.byref(_ins()), C.byref(_ins()), None, None, P + 0x604, P + 0x800, None, None) == 3
+    # a block whose checkpoints fit neither long mode (bf16, N = 16: K > 1392 and K > 768)
+    d = Dims(1, 2048, 64, 16, 2048, 1, 1)
+    assert f(C.byref(d), C.byref(_ins()), C.byref(_ins()), None, None, P + 0x600, P + 0x800, None, None) == 2
+
+
+@cpu_only
+@pytest.mark.parametrize("noalloc", [False, True])
+def test_prefill_chunked_checks_both_passes_first(lib, noalloc):
+    lib.bdscan_prefill_chunked.argtypes = [C.POINTER(Dims), C.POINTER(Inputs)] + [C.c_void_p] * 5 + \
+        [C.c_size_t, C.c_void_p]
+    lib.bdscan_prefill_chunked_noalloc.argtypes = [C.POINTER(Dims), C.POINTER(Inputs)] + [C.c_void_p] * 5
+    lib.bdscan_prefill_chunked_workspace.argtypes = [C.POINTER(Dims)]
+    lib.bdscan_prefill_chunked_workspace.restype = C.c_size_t
+    d = Dims(1, 65536, 1536, 16, 32, 1, 1)   # one sequence: 48 rows, so the chunked path runs
+    assert lib.bdscan_prefill_chunked_workspace(C.byref(d)) > 0
+
+    def call(h0, y, h_out, bnd):
+        if noalloc:
+            return lib.bdscan_prefill_chunked_noalloc(C.byref(d), C.byref(_ins()), h0, y, h_out, bnd, None)
+        return lib.bdscan_prefill_chunked(C.byref(d), C.byref(_ins()), h0, y, h_out, bnd, P + 0x9000, 1 << 30,
+                                          None)
+    assert call(None, P + 0x600, None, None) == 1                 # h_out required by pass 2
+    assert call(None, P + 0x604, P + 0x700, None) == 3            # y misaligned
+    assert call(P + 0x808, P + 0x600, P + 0x700, None) == 3       # h0 misaligned
+    assert call(None, P + 0x600, P + 0x700, P + 0x90c) == 3       # boundary misaligned
