@@ -1,18 +1,23 @@
 #!/usr/bin/env python
 """Benchmark of the block-confined bidirectional selective scan on B200.
 
-One step = one full-block (all-block) training pass of the mixer over one batch
-of synthetic input: the forward scan over every token, the reverse scan inside
-every block, the fused softplus / exp / skip / combine, and the block-boundary
-cache states (every row of the hot path). The default workload is the training
-configuration: batch 8, L 4096, D 1536, N 16, block 16, bf16 I/O, fp32 state.
+One step = one pass of the mixer's hot path through every layer of the
+350M-scale stack: 24 layers, each a full-block (all-block) pass over batch 16 x
+8192 tokens x 2048 channels with N = 64 and blocks of 16 tokens (the forward
+scan over every token, the reverse scan inside every block, the fused softplus
+/ exp / skip / combine), bf16 I/O, fp32 state. This is the largest workload that
+fits one GPU; per-layer A and Dskip, x/dt/B/C shared by the layers.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 Prints one JSON line (rank 0). Under torchrun every rank runs its own batch
 (independent sequences, no data-path collective: weak scaling); the timing is
-the max over ranks. `--impl reference` times the fp64 CPU oracle instead, on a
-bounded sample of the same workload.
+the max over ranks. Besides the headline, the line carries (one GPU only) the
+other block sizes of the stack and `secondary` records: the training workload
+(batch 8 x 4096 x 1536, N = 16) forward and backward, and the 65,536- and
+262,144-token inference workloads (prefill, block step, graph-replayed block
+loop, full-sequence comparator). `--impl reference` times the fp64 CPU oracle
+instead, on a bounded sample of the same workload.
 """
 from __future__ import annotations
 
@@ -33,11 +38,15 @@ sys.path.insert(0, ROOT)
 
 from selective_ssm_scan_mamba_b200 import inputs as I  # noqa: E402
 
-WORKLOAD = "train"
+WORKLOAD = "stack350m"
+STACK_K = 16                 # headline block size of the stack (the others are sub-results)
+ORACLE_SAMPLE_CHANNELS = 128  # oracle sample of the stack: one layer, all sequences, these channels
 METRIC = "bidirectional block-scan tokens/s and achieved HBM GB/s vs B200 peak"
 SM_COUNT = 148
-EX2_PER_CLK_SM = 16          # MUFU.EX2 results per clock per SM (measured 15.9 on this machine)
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "train_traffic.json")
+EX2_PER_CLK_SM = 16          # MUFU.EX2 results per clock per SM: the nominal rate of the special-function
+                             # unit (a throughput probe on this machine measured 15.9; not in the driver's peaks)
+PROFILE_TRAFFIC = {"stack350m": os.path.join(ROOT, "profiles", "stack350m_traffic.json"),
+                   "train": os.path.join(ROOT, "profiles", "train_traffic.json")}
 
 
 def kernel_source_hash() -> str:
@@ -149,24 +158,38 @@ def max_over_ranks(values, device=None):
     return [float(v) for v in t]
 
 
-def job_tokens_per_step(w, world: int) -> int:
-    return w.batch * w.L * world
+def stack_tokens_per_step(w, world: int) -> int:
+    """Token-layers per step of the stack: every layer scans every token of every sequence."""
+    return w.batch * w.L * w.layers * world
+
+
+def config_dict(w, world: int, K: int) -> dict:
+    """The workload named in both arms' JSON lines (identical keys and values)."""
+    return {"workload": w.name, "batch": w.batch, "seq_len": w.L, "d_inner": w.D, "d_state": w.N,
+            "layers": w.layers, "block": K, "io_dtype": w.io, "state_dtype": "f32",
+            "outputs": "y of every layer", "count": "tokens x layers (each layer scans every token)",
+            "parallelism": f"dp{world}",
+            "l2": "working set 1.64 GB per layer launch > 126 MB L2 (no flush)"}
+
+
+def _up(a, dev=None, pin=False):
+    """numpy array (bf16 as uint16 bits) -> torch tensor on dev, or pinned host memory."""
+    import torch
+    a = np.ascontiguousarray(a)
+    t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+    return t.pin_memory() if pin else t.to(dev)
 
 
 # ------------------------------------------------------------------ CPU oracle
-def _oracle_worker(conn, name, seed, n_seq, c0, c1):
-    """One process of OraclePool: regenerates its channel slice of the workload
-    once, then runs the oracle on it whenever asked."""
+def _oracle_worker(conn):
+    """One process of OraclePool: receives its channel slice once, then runs
+    the oracle's full-block pass on it whenever asked."""
     import oracle
-    w = I.WORKLOADS[name]
-    chans = list(range(c0, c1))
-    s = I.make_sequence(seed, n_seq, w.L, w.D, w.N, w.io, channels=chans)
-    p = I.make_params(seed, w.D, w.N)
-    A, Dk = p["A"][c0:c1].copy(), p["Dskip"][c0:c1].copy()
     oracle.load()
+    job = conn.recv()
     conn.send("ready")
     while conn.recv() == "run":
-        oracle.train_blocks(s["x"], s["dt"], A, s["B"], s["C"], Dk, w.K)
+        oracle.train_blocks(job["x"], job["dt"], job["A"], job["B"], job["C"], job["Dskip"], job["K"])
         conn.send("done")
 
 
@@ -183,21 +206,25 @@ def cpu_model() -> str:
 
 class OraclePool:
     """The fp64 oracle, unchanged, on every host core: `workers` spawned
-    processes each own a contiguous slice of the channels (channels are
-    independent in the scan) of the first n_seq sequences; a step runs all
-    slices at once and its time is the wall-clock time until the last is done."""
+    processes each own a contiguous slice of the given channels (channels are
+    independent in the scan); a step runs all slices at once and its time is
+    the wall-clock time until the last is done. s: x, dt [n_seq, L, channels],
+    B, C [n_seq, L, N]; A [channels, N], Dskip [channels]."""
 
-    def __init__(self, w, seed, n_seq, workers=None):
+    def __init__(self, s, A, Dskip, K, workers=None):
         import multiprocessing as mp
-        self.w, self.n_seq = w, n_seq
-        self.workers = max(1, min(workers or os.cpu_count() or 1, w.D))
+        nch = s["x"].shape[2]
+        self.workers = max(1, min(workers or os.cpu_count() or 1, nch))
         ctx = mp.get_context("spawn")
         self.conns, self.procs = [], []
         for i in range(self.workers):
-            c0, c1 = i * w.D // self.workers, (i + 1) * w.D // self.workers
+            c0, c1 = i * nch // self.workers, (i + 1) * nch // self.workers
             a, b = ctx.Pipe()
-            pr = ctx.Process(target=_oracle_worker, args=(b, w.name, seed, n_seq, c0, c1), daemon=True)
+            pr = ctx.Process(target=_oracle_worker, args=(b,), daemon=True)
             pr.start()
+            a.send({"x": np.ascontiguousarray(s["x"][:, :, c0:c1]), "dt": np.ascontiguousarray(s["dt"][:, :, c0:c1]),
+                    "B": s["B"], "C": s["C"], "A": np.ascontiguousarray(A[c0:c1]),
+                    "Dskip": np.ascontiguousarray(Dskip[c0:c1]), "K": K})
             self.conns.append(a)
             self.procs.append(pr)
         for c in self.conns:
@@ -211,9 +238,6 @@ class OraclePool:
             c.recv()
         return time.perf_counter() - t0
 
-    def tokens_per_step(self) -> int:
-        return self.n_seq * self.w.L
-
     def close(self):
         for c in self.conns:
             c.send("stop")
@@ -221,35 +245,83 @@ class OraclePool:
             pr.join(timeout=30)
 
 
+def stack_oracle_pool(w, seed, K):
+    """The oracle on the bounded sample of the stack: layer 0, all sequences,
+    all tokens, channels [0, ORACLE_SAMPLE_CHANNELS). The scan's cost is exactly
+    linear in channels and layers, so a sample time t stands for
+    t * (D / channels) * layers of the whole step."""
+    chans = list(range(ORACLE_SAMPLE_CHANNELS))
+    s = I.make_sequence(seed, w.batch, w.L, w.D, w.N, w.io, channels=chans)
+    p = I.make_params(w.seed, w.D, w.N, layer=0)
+    pool = OraclePool(s, p["A"][:len(chans)], p["Dskip"][:len(chans)], K)
+    sample = (f"one layer, all {w.batch} sequences x {w.L} tokens, channels 0-{len(chans) - 1} of {w.D}, "
+              f"block {K}, split over {pool.workers} processes; extrapolated linearly to {w.D} channels "
+              f"and {w.layers} layers")
+    return pool, sample
+
+
+def oracle_value(w, secs: float) -> float:
+    """Stack tokens x layers per second implied by one sample time."""
+    full_step = secs * (w.D / ORACLE_SAMPLE_CHANNELS) * w.layers
+    return w.batch * w.L * w.layers / full_step
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     w = I.WORKLOADS[WORKLOAD]
-    pool = OraclePool(w, w.seed, w.batch)
+    pool, sample = stack_oracle_pool(w, w.seed, STACK_K)
     try:
         for _ in range(args.warmup):
             pool.step()
         times = [pool.step() for _ in range(args.steps)]
     finally:
         pool.close()
-    per_step = statistics.mean(times)
-    value = pool.tokens_per_step() / per_step
-    sample = (f"all {w.batch} sequences x {w.L} tokens x {w.D} channels per step, channels split over "
-              f"{pool.workers} processes")
+    per_sample = statistics.mean(times)
+    value = oracle_value(w, per_sample)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "warmup": args.warmup, "ms_per_step": w.batch * w.L * w.layers / value * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
-        "config": {"workload": WORKLOAD, "batch": w.batch, "seq_len": w.L, "d_inner": w.D, "d_state": w.N,
-                   "block": w.K, "io_dtype": w.io, "parallelism": f"dp{args.gpus}", "sample": sample},
+        "config": config_dict(w, args.gpus, STACK_K),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": pool.workers, "kind": "oracle",
-                         "sample": sample, "cpu": cpu_model()},
+                         "sample": sample, "sample_s": per_sample, "cpu": cpu_model()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def traffic_for(workload: str):
+    """ncu DRAM bytes per launch recorded for the kernel, if the kernel's code is
+    unchanged since the capture (else None)."""
+    path = PROFILE_TRAFFIC.get(workload)
+    if path and os.path.exists(path):
+        pt = json.load(open(path))
+        if pt.get("kernel_source_hash") == kernel_source_hash():
+            return pt.get("traffic_bytes_per_launch")
+    return None
+
+
+def ex2_peak_g(peaks) -> float:
+    return EX2_PER_CLK_SM * SM_COUNT * peaks["sm_max_mhz"] * 1e-3
+
+
+def roofline(elem_steps: int, nbytes: int, launch_ms: float, peaks, traffic=None, kernel="") -> dict:
+    """SFU roofline of one launch (one MUFU.EX2 per element-step) with the HBM
+    fraction of its algorithmic bytes beside it."""
+    rate = elem_steps / (launch_ms * 1e-3) / 1e9
+    gbs = nbytes / (launch_ms * 1e-3) / 1e9
+    return {"bound": "alu", "achieved": rate, "peak": ex2_peak_g(peaks), "unit": "Gex2/s",
+            "frac": rate / ex2_peak_g(peaks), "traffic": traffic,
+            "peak_source": f"nominal {EX2_PER_CLK_SM} MUFU.EX2/clk/SM x {SM_COUNT} SMs x "
+                           f"{peaks['sm_max_mhz']:.0f} MHz (probe on this pool: 15.9/clk/SM)",
+            "hbm": {"achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                    "peak_source": peaks["source"], "frac_of_nominal_8000": gbs / 8000.0,
+                    "algorithmic_bytes_per_launch": nbytes},
+            "ex2_per_launch": elem_steps, "kernel": kernel, "kernel_ms": launch_ms}
 
 
 # ------------------------------------------------------------------ GPU path
@@ -270,101 +342,115 @@ def run_ours(args):
     from selective_ssm_scan_mamba_b200 import bdscan
 
     w = I.WORKLOADS[WORKLOAD]
+    K = STACK_K
     seed = rank_seed(w.seed, rank)
     s = I.make_sequence(seed, w.batch, w.L, w.D, w.N, w.io)
-    p = I.make_params(w.seed, w.D, w.N)
-
-    def up(a, pin=False):
-        a = np.ascontiguousarray(a)
-        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
-        return t.pin_memory() if pin else t.to(dev)
-
-    g = {k: up(v) for k, v in s.items()}
-    A, Dk = up(p["A"]), up(p["Dskip"])
+    params = [I.make_params(w.seed, w.D, w.N, layer=l) for l in range(w.layers)]
+    g = {k: _up(v, dev) for k, v in s.items()}
+    As = [_up(q["A"], dev) for q in params]
+    Ds = [_up(q["Dskip"], dev) for q in params]
     y = torch.empty((w.batch, w.L, w.D), dtype=torch.bfloat16, device=dev)
-    bnd = torch.empty((w.batch, w.L // w.K, w.D, w.N), dtype=torch.float32, device=dev)
-    hout = torch.empty((w.batch, w.D, w.N), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        bdscan.train_blocks(g["x"], g["dt"], A, g["B"], g["C"], Dk, w.K, y=y, boundary=bnd, h_out=hout)
+    def layers(inp, yout, Kb, evs=None):
+        for l in range(w.layers):
+            if evs is not None:
+                evs[l][0].record(stream)
+            bdscan.train_blocks(inp["x"], inp["dt"], As[l], inp["B"], inp["C"], Ds[l], Kb, y=yout)
+            if evs is not None:
+                evs[l][1].record(stream)
 
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local])
 
-    for _ in range(max(args.warmup, 3)):
-        step()
+    warm = max(args.warmup, 3)
+    for _ in range(warm):
+        layers(g, y, K)
     torch.cuda.synchronize(dev)
 
     # timed region: device time with CUDA events on the launching stream; one
-    # event pair per launch gives the per-launch duration for the roofline.
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # event pair per layer launch gives the per-launch duration for the roofline
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(w.layers)]
+          for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         barrier()
         torch.cuda.synchronize(dev)
         start.record(stream)
         for i in range(args.steps):
-            ev[i][0].record(stream)
-            step()
-            ev[i][1].record(stream)
+            layers(g, y, K, ev[i])
         stop.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
     elapsed_ms, launch_ms = max_over_ranks(
-        [start.elapsed_time(stop), statistics.mean(a.elapsed_time(b) for a, b in ev)], device=dev)
+        [start.elapsed_time(stop), statistics.mean(a.elapsed_time(b) for st in ev for a, b in st)], device=dev)
     ms_per_step = elapsed_ms / args.steps
-    tokens_per_step = job_tokens_per_step(w, world)
+    tokens_per_step = stack_tokens_per_step(w, world)
     value = tokens_per_step / (ms_per_step * 1e-3)
+    peaks = load_peaks()
+    elem = w.batch * w.L * w.D * w.N
+    nbytes = algorithmic_bytes(w, boundary=False, h_out=False)
+    roof = roofline(elem, nbytes, launch_ms, peaks, traffic_for("stack350m"),
+                    kernel=f"bdscan_kernel<bf16, N=64, fused, K={K}>")
 
-    # end to end through the public call with host buffers: every step copies its
-    # inputs from pinned host memory, runs the pass and reads all its outputs
-    # (y, boundary states, final state) back into pinned host memory. Steps are
-    # pipelined on three streams with two device buffer sets: step k's upload
-    # overlaps step k-1's pass and step k-2's download (PCIe is full duplex).
-    hx = {k: up(v, pin=True) for k, v in s.items()}
-    hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    hb = torch.empty(bnd.shape, dtype=bnd.dtype).pin_memory()
-    hh = torch.empty(hout.shape, dtype=hout.dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in hx.values())
-    d2h = hy.numel() * hy.element_size() + hb.numel() * hb.element_size() + hh.numel() * hh.element_size()
-    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    s_c = stream
-    bufs = []
-    for i in range(2):
-        bufs.append({"in": {k: torch.empty_like(v, device=dev) for k, v in hx.items()},
-                     "y": y if i == 0 else torch.empty_like(y), "bnd": bnd if i == 0 else torch.empty_like(bnd),
-                     "hout": hout if i == 0 else torch.empty_like(hout),
-                     "ev_in": torch.cuda.Event(), "ev_c": torch.cuda.Event(), "ev_out": torch.cuda.Event()})
+    # the other block sizes of the stack (same inputs, 24 layers each)
+    by_block = {str(K): {"ms_24_layers": ms_per_step, "tokens_per_s": value / world, "sfu_frac": roof["frac"],
+                         "hbm_frac": roof["hbm"]["frac"]}}
+    for Kb in (k for k in I.STACK_BLOCK_SIZES if k != K):
+        layers(g, y, Kb)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 2
+        e0.record(stream)
+        for _ in range(reps):
+            layers(g, y, Kb)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / reps
+        per_layer = ms / w.layers
+        by_block[str(Kb)] = {"ms_24_layers": ms, "tokens_per_s": w.batch * w.L * w.layers / (ms * 1e-3),
+                             "sfu_frac": elem / (per_layer * 1e-3) / 1e9 / ex2_peak_g(peaks),
+                             "hbm_frac": nbytes / (per_layer * 1e-3) / 1e9 / peaks["hbm_gbs"]}
 
-    def e2e_steps_run(n):
-        for k in range(n):
-            bf = bufs[k % 2]
-            with torch.cuda.stream(s_in):
-                if k >= 2:
-                    s_in.wait_event(bf["ev_c"])        # the pass two steps back has read these inputs
-                for name in hx:
-                    bf["in"][name].copy_(hx[name], non_blocking=True)
-                bf["ev_in"].record(s_in)
-            with torch.cuda.stream(s_c):
-                s_c.wait_event(bf["ev_in"])
-                if k >= 2:
-                    s_c.wait_event(bf["ev_out"])       # the download two steps back has read these outputs
-                d = bf["in"]
-                bdscan.train_blocks(d["x"], d["dt"], A, d["B"], d["C"], Dk, w.K, y=bf["y"], boundary=bf["bnd"],
-                                    h_out=bf["hout"])
-                bf["ev_c"].record(s_c)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(bf["ev_c"])
-                hy.copy_(bf["y"], non_blocking=True)
-                hb.copy_(bf["bnd"], non_blocking=True)
-                hh.copy_(bf["hout"], non_blocking=True)
-                bf["ev_out"].record(s_out)
-
-    e2e_value = None
+    # end to end through the public call with host buffers: every step copies
+    # x, dt, B, C from pinned host memory, runs the 24 layers and reads the last
+    # layer's y back into pinned host memory. Steps are pipelined on three
+    # streams with two device buffer sets: step k's upload overlaps step k-1's
+    # layers and step k-2's download (PCIe is full duplex).
+    e2e_value, h2d, d2h = None, 0, 0
     if not args.no_e2e:
-        e2e_steps = max(2, min(args.steps, 8))
+        hx = {k: _up(v, pin=True) for k, v in s.items()}
+        hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in hx.values())
+        d2h = hy.numel() * hy.element_size()
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        bufs = []
+        for i in range(2):
+            bufs.append({"in": {k: torch.empty_like(v, device=dev) for k, v in hx.items()},
+                         "y": y if i == 0 else torch.empty_like(y),
+                         "ev_in": torch.cuda.Event(), "ev_c": torch.cuda.Event(), "ev_out": torch.cuda.Event()})
+
+        def e2e_steps_run(n):
+            for k in range(n):
+                bf = bufs[k % 2]
+                with torch.cuda.stream(s_in):
+                    if k >= 2:
+                        s_in.wait_event(bf["ev_c"])        # the layers two steps back have read these inputs
+                    for name in hx:
+                        bf["in"][name].copy_(hx[name], non_blocking=True)
+                    bf["ev_in"].record(s_in)
+                stream.wait_event(bf["ev_in"])
+                if k >= 2:
+                    stream.wait_event(bf["ev_out"])        # the download two steps back has read this y
+                layers(bf["in"], bf["y"], K)
+                bf["ev_c"].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(bf["ev_c"])
+                    hy.copy_(bf["y"], non_blocking=True)
+                    bf["ev_out"].record(s_out)
+
+        e2e_steps = max(2, min(args.steps, 6))
         e2e_steps_run(2)
         torch.cuda.synchronize(dev)
         barrier()
@@ -375,57 +461,88 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         (te,) = max_over_ranks([e0.elapsed_time(e1)], device=dev)
         e2e_value = tokens_per_step / (te / e2e_steps * 1e-3)
-
-    peaks = load_peaks()
-    nbytes = algorithmic_bytes(w)
-    hbm_gbs = nbytes / (launch_ms * 1e-3) / 1e9
-    ex2 = w.batch * w.L * w.D * w.N
-    ex2_rate = ex2 / (launch_ms * 1e-3) / 1e9
-    ex2_peak = EX2_PER_CLK_SM * SM_COUNT * peaks["sm_max_mhz"] * 1e6 / 1e9
-    traffic = None
-    if os.path.exists(PROFILE_TRAFFIC):
-        pt = json.load(open(PROFILE_TRAFFIC))
-        if pt.get("kernel_source_hash") == kernel_source_hash():
-            traffic = pt.get("traffic_bytes_per_launch")
+        del bufs, hx, hy
     clocks = clk.summary()
+    del g
+    torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        pool = OraclePool(w, w.seed, w.batch)
+        pool, sample = stack_oracle_pool(w, w.seed, K)
         try:
             secs = pool.step()
         finally:
             pool.close()
-        cpu = {"value": pool.tokens_per_step() / secs, "unit": "tokens/s", "cores": pool.workers, "kind": "oracle",
-               "sample": f"all {w.batch} sequences x {w.L} tokens x {w.D} channels once, channels split over "
-                         f"{pool.workers} processes, {secs:.1f} s", "cpu": cpu_model()}
+        cpu = {"value": oracle_value(w, secs), "unit": "tokens/s", "cores": pool.workers, "kind": "oracle",
+               "sample": f"{sample}; {secs:.1f} s", "cpu": cpu_model()}
+
+    secondary = None
+    if world == 1 and not args.no_secondary:
+        secondary = {}
+        for name, fn in (("train", lambda: measure_train(dev, peaks, 20, 5)),
+                         ("train_fwd_bwd", lambda: measure_train_step(dev, peaks, 5, 3)),
+                         ("step65k", lambda: measure_inference("step65k", dev, peaks)),
+                         ("step262k", lambda: measure_inference("step262k", dev, peaks))):
+            try:
+                secondary[name] = fn()
+            except Exception as e:   # reported in the line, the headline stands
+                secondary[name] = {"error": f"{type(e).__name__}: {e}"}
+            torch.cuda.empty_cache()
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": warm, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "batch": w.batch, "seq_len": w.L, "d_inner": w.D, "d_state": w.N,
-                   "block": w.K, "io_dtype": w.io, "state_dtype": "f32", "outputs": "y + all block-boundary states + final state",
-                   "parallelism": f"dp{world}", "l2": "working set 506 MB per step > 126 MB L2 (no flush)"},
-        "roofline": {"bound": "alu", "achieved": ex2_rate, "peak": ex2_peak, "unit": "Gex2/s",
-                     "frac": ex2_rate / ex2_peak, "traffic": traffic,
-                     "peak_source": f"16 MUFU.EX2/clk/SM x {SM_COUNT} SMs x {peaks['sm_max_mhz']:.0f} MHz",
-                     "hbm": {"achieved": hbm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                             "frac": hbm_gbs / peaks["hbm_gbs"], "peak_source": peaks["source"],
-                             "frac_of_nominal_8000": hbm_gbs / 8000.0,
-                             "algorithmic_bytes_per_launch": nbytes},
-                     "kernel_ms": launch_ms},
+        "config": config_dict(w, world, K),
+        "roofline": roof,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * w.layers,
         "clocks": clocks,
+        "by_block": by_block,
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
+    if secondary is not None:
+        line["secondary"] = secondary
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+def measure_train(dev, peaks, steps=20, warmup=5) -> dict:
+    """The training workload (batch 8 x 4096 x 1536, N = 16, K = 16): one
+    full-block pass writing y, every block-boundary state and the final state."""
+    import torch
+    from selective_ssm_scan_mamba_b200 import bdscan
+    w = I.WORKLOADS["train"]
+    s = I.make_sequence(w.seed, w.batch, w.L, w.D, w.N, w.io)
+    p = I.make_params(w.seed, w.D, w.N)
+    g = {k: _up(v, dev) for k, v in s.items()}
+    A, Dk = _up(p["A"], dev), _up(p["Dskip"], dev)
+    y = torch.empty((w.batch, w.L, w.D), dtype=torch.bfloat16, device=dev)
+    bnd = torch.empty((w.batch, w.L // w.K, w.D, w.N), dtype=torch.float32, device=dev)
+    hout = torch.empty((w.batch, w.D, w.N), dtype=torch.float32, device=dev)
+
+    def step():
+        bdscan.train_blocks(g["x"], g["dt"], A, g["B"], g["C"], Dk, w.K, y=y, boundary=bnd, h_out=hout)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
+        a.record()
+        step()
+        b.record()
+    torch.cuda.synchronize(dev)
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    return {"config": {"batch": w.batch, "seq_len": w.L, "d_inner": w.D, "d_state": w.N, "block": w.K,
+                       "io_dtype": w.io, "outputs": "y + all block-boundary states + final state"},
+            "ms": ms, "tokens_per_s": w.batch * w.L / (ms * 1e-3),
+            "roofline": roofline(w.batch * w.L * w.D * w.N, algorithmic_bytes(w), ms, peaks, traffic_for("train"),
+                                 kernel="bdscan_kernel<bf16, N=16, fused, K=16>")}
 
 
 # ------------------------------------------------------- inference workloads
@@ -446,26 +563,20 @@ def prefill_bytes(w, L) -> int:
     return w.batch * L * w.D * 3 * s + w.batch * L * w.N * 2 * s + 4 * w.D * w.N + 4 * w.D + 4 * w.batch * w.D * w.N
 
 
-def run_inference(args, name):
+def measure_inference(name, dev, peaks) -> dict:
     """Block-diffusion inference at a long context: prefill (forward-only scan of
     the context), then per block `steps` denoising steps (forward from the cache
     plus in-block reverse) and one commit. Reports the prefill, the single step
-    (inputs from a rotating pool larger than twice L2, so they come from HBM) and
-    the whole denoise loop replayed as a CUDA graph."""
+    (inputs from a rotating pool larger than twice L2, so they come from HBM;
+    device time and the host time of an eager call through the binding) and the
+    whole denoise loop replayed as a CUDA graph."""
     import torch
     from selective_ssm_scan_mamba_b200 import bdscan
     w = I.WORKLOADS[name]
-    dev = torch.device("cuda", 0)
-    peaks = load_peaks()
     L, K = w.L, w.K
-
-    def up(a):
-        a = np.ascontiguousarray(a)
-        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
-        return t.to(dev)
-
+    sfu = ex2_peak_g(peaks)
     p = I.make_params(w.seed, w.D, w.N)
-    A, Dk = up(p["A"]), up(p["Dskip"])
+    A, Dk = _up(p["A"], dev), _up(p["Dskip"], dev)
     ctx = {k: torch.empty((w.batch, L, w.D if k in ("x", "dt") else w.N), dtype=torch.bfloat16, device=dev)
            for k in ("x", "dt", "B", "C")}
     span = 8 * I.CHUNK
@@ -473,7 +584,7 @@ def run_inference(args, name):
         n = min(span, L - t0)
         sq = I.make_sequence(w.seed, w.batch, n, w.D, w.N, w.io, stream=("context",), t0=t0)
         for k in ctx:
-            ctx[k][:, t0:t0 + n] = up(sq[k])
+            ctx[k][:, t0:t0 + n] = _up(sq[k], dev)
     y_ctx = torch.empty((w.batch, L, w.D), dtype=torch.bfloat16, device=dev)
     cache = torch.empty((w.batch, w.D, w.N), dtype=torch.float32, device=dev)
 
@@ -501,6 +612,7 @@ def run_inference(args, name):
 
     prefill_seq_ms = timed(prefill)
     prefill_ms = timed(prefill_chunked)
+    chunked = int(ws.numel()) > 16
 
     # rotating pool of noisy block inputs, > 2x L2
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -508,9 +620,9 @@ def run_inference(args, name):
     pool_n = max(64, int(2.2 * l2 / per) + 1)
     total_steps = w.blocks * w.steps
     nz = I.make_sequence(w.seed, w.batch, K * pool_n, w.D, w.N, w.io, stream=("noisy", 0, 0))
-    pool = {k: up(v).view(w.batch, pool_n, K, -1).transpose(0, 1).contiguous() for k, v in nz.items()}
+    pool = {k: _up(v, dev).view(w.batch, pool_n, K, -1).transpose(0, 1).contiguous() for k, v in nz.items()}
     cl = I.make_sequence(w.seed, w.batch, K * w.blocks, w.D, w.N, w.io, stream=("context",), t0=L)
-    clean = {k: up(v).view(w.batch, w.blocks, K, -1).transpose(0, 1).contiguous() for k, v in cl.items()}
+    clean = {k: _up(v, dev).view(w.batch, w.blocks, K, -1).transpose(0, 1).contiguous() for k, v in cl.items()}
     y_step = torch.empty((w.batch, K, w.D), dtype=torch.bfloat16, device=dev)
 
     def step(i):
@@ -528,6 +640,17 @@ def run_inference(args, name):
         evs[i][1].record()
     torch.cuda.synchronize(dev)
     step_us = statistics.median(a.elapsed_time(b) for a, b in evs) * 1e3
+    # host cost of an eager call through the Python binding (argument checks,
+    # marshalling, launch), the step's inputs prepared beforehand
+    qs = [{k: v[i % pool_n] for k, v in pool.items()} for i in range(200)]
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    for q in qs:
+        bdscan.block_step(q["x"], q["dt"], A, q["B"], q["C"], Dk, cache, y=y_step)
+    host_us = (time.perf_counter() - t0) / len(qs) * 1e6
+    torch.cuda.synchronize(dev)
+    eager_us = (time.perf_counter() - t0) / len(qs) * 1e6
+    del qs
 
     # the whole denoise loop (all blocks: steps + commit) as one CUDA graph
     cache0 = cache.clone()
@@ -557,12 +680,16 @@ def run_inference(args, name):
     loop_ms = statistics.median(loop_ms)
     del g
     launches = total_steps + w.blocks
+    loop_bytes = total_steps * per + w.blocks * commit_bytes(w)
+    loop_elem = (total_steps + w.blocks) * w.batch * K * w.D * w.N
 
     # the full-sequence bidirectional comparator: one denoising step re-runs
     # the reverse scan over the whole context + block (DiffuMamba-style mixing)
     full_ms = None
     if w.batch * (L + K) * w.D * 2 * 3 < 40e9:
-        fx = {k: torch.cat([ctx[k], pool[k][0]], dim=1).contiguous() for k in ctx}
+        del pool
+        fx = {k: torch.cat([ctx[k], clean[k][0]], dim=1).contiguous() for k in ctx}
+        del ctx, y_ctx
         fy = torch.empty((w.batch, L + K, w.D), dtype=torch.bfloat16, device=dev)
 
         def full_step():
@@ -577,77 +704,37 @@ def run_inference(args, name):
         torch.cuda.synchronize(dev)
         full_ms = e0.elapsed_time(e1) / 3
         del fx, fy
-    line = {
-        "metric": METRIC, "workload": name, "n_gpus": 1, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": name, "batch": w.batch, "context": L, "d_inner": w.D, "d_state": w.N, "block": K,
+    pf_elem = w.batch * L * w.D * w.N
+    pf_bytes = prefill_bytes(w, L)
+    return {
+        "config": {"batch": w.batch, "context": L, "d_inner": w.D, "d_state": w.N, "block": K,
                    "steps_per_block": w.steps, "blocks": w.blocks, "io_dtype": w.io},
-        "prefill": {"ms": prefill_ms, "kind": "time-chunked (bdscan_prefill_chunked)",
-                    "sequential_ms": prefill_seq_ms, "workspace_bytes": int(ws.numel()),
+        "prefill": {"ms": prefill_ms,
+                    "kind": "time-chunked (bdscan_prefill_chunked)" if chunked else
+                            "sequential (bdscan_prefill_chunked runs the sequential scan: enough rows)",
+                    "sequential_ms": prefill_seq_ms, "workspace_bytes": int(ws.numel()) if chunked else 0,
                     "tokens_per_s": w.batch * L / (prefill_ms * 1e-3),
-                    "hbm_gbs": prefill_bytes(w, L) / (prefill_ms * 1e-3) / 1e9,
-                    "hbm_frac": prefill_bytes(w, L) / (prefill_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                    "ex2_frac": w.batch * L * w.D * w.N / (prefill_ms * 1e-3) / 1e9 /
-                                (EX2_PER_CLK_SM * SM_COUNT * peaks["sm_max_mhz"] * 1e-3)},
+                    "algorithmic_bytes": pf_bytes,
+                    "hbm_gbs": pf_bytes / (prefill_ms * 1e-3) / 1e9,
+                    "hbm_frac": pf_bytes / (prefill_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                    "sfu_frac": pf_elem / (prefill_ms * 1e-3) / 1e9 / sfu},
         "step": {"us": step_us, "scanned_tokens_per_s": w.batch * K / (step_us * 1e-6),
                  "algorithmic_bytes": per, "hbm_gbs": per / (step_us * 1e-6) / 1e9,
                  "hbm_frac": per / (step_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                 "sfu_frac": w.batch * K * w.D * w.N / (step_us * 1e-6) / 1e9 / sfu,
+                 "eager_call_us": eager_us, "eager_host_us": host_us,
                  "inputs": f"rotating pool of {pool_n} step inputs ({pool_n * per / 1e6:.0f} MB > 2x L2)"},
         "loop": {"ms": loop_ms, "graph_launches": launches, "us_per_launch": loop_ms * 1e3 / launches,
                  "committed_tokens_per_s": w.batch * K * w.blocks / (loop_ms * 1e-3),
                  "scanned_tokens_per_s": w.batch * K * launches / (loop_ms * 1e-3),
-                 "hbm_gbs": (total_steps * per + w.blocks * commit_bytes(w)) / (loop_ms * 1e-3) / 1e9},
+                 "hbm_gbs": loop_bytes / (loop_ms * 1e-3) / 1e9,
+                 "hbm_frac": loop_bytes / (loop_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                 "sfu_frac": loop_elem / (loop_ms * 1e-3) / 1e9 / sfu},
         "full_sequence_step": None if full_ms is None else {
             "ms": full_ms, "tokens": L + K,
             "vs_block_step": full_ms * 1e3 / step_us,
             "note": "forward + reverse scan over context + active block per denoising step"},
     }
-    print(json.dumps(line), flush=True)
-    return 0
-
-
-def run_stack(args):
-    """24-layer N = 64 stack: one full-block pass per layer (per-layer A, Dskip),
-    for each block size; tokens/s = batch * L * layers / time."""
-    import torch
-    from selective_ssm_scan_mamba_b200 import bdscan
-    w = I.WORKLOADS["stack350m"]
-    dev = torch.device("cuda", 0)
-    peaks = load_peaks()
-
-    def up(a):
-        a = np.ascontiguousarray(a)
-        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
-        return t.to(dev)
-
-    s = I.make_sequence(w.seed, w.batch, w.L, w.D, w.N, w.io)
-    g = {k: up(v) for k, v in s.items()}
-    params = [I.make_params(w.seed, w.D, w.N, layer=l) for l in range(w.layers)]
-    As = [up(q["A"]) for q in params]
-    Ds = [up(q["Dskip"]) for q in params]
-    y = torch.empty((w.batch, w.L, w.D), dtype=torch.bfloat16, device=dev)
-    res = {}
-    for K in I.STACK_BLOCK_SIZES:
-        def layers():
-            for l in range(w.layers):
-                bdscan.train_blocks(g["x"], g["dt"], As[l], g["B"], g["C"], Ds[l], K, y=y)
-        layers()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        layers()
-        e1.record()
-        torch.cuda.synchronize(dev)
-        ms = e0.elapsed_time(e1)
-        per_layer = ms / w.layers
-        res[str(K)] = {"ms_24_layers": ms, "tokens_per_s": w.batch * w.L * w.layers / (ms * 1e-3),
-                       "ex2_frac": w.batch * w.L * w.D * w.N / (per_layer * 1e-3) / 1e9 /
-                                   (EX2_PER_CLK_SM * SM_COUNT * peaks["sm_max_mhz"] * 1e-3),
-                       "hbm_frac": algorithmic_bytes(w, boundary=False, h_out=False) / (per_layer * 1e-3) / 1e9
-                                   / peaks["hbm_gbs"]}
-    print(json.dumps({"metric": METRIC, "workload": "stack350m", "config": {"batch": w.batch, "seq_len": w.L,
-                      "d_inner": w.D, "d_state": w.N, "layers": w.layers, "io_dtype": w.io},
-                      "by_block": res}), flush=True)
-    return 0
 
 
 def backward_bytes(w) -> int:
@@ -662,25 +749,17 @@ def backward_bytes(w) -> int:
     return n
 
 
-def run_train_step(args):
-    """Training step of the headline workload: the all-block forward pass
+def measure_train_step(dev, peaks, steps=5, warmup=3) -> dict:
+    """Training step of the training workload: the all-block forward pass
     (y + block-boundary states) and its backward pass given dy."""
     import torch
     from selective_ssm_scan_mamba_b200 import bdscan
     w = I.WORKLOADS["train"]
-    dev = torch.device("cuda", 0)
-    peaks = load_peaks()
-
-    def up(a):
-        a = np.ascontiguousarray(a)
-        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
-        return t.to(dev)
-
     s = I.make_sequence(w.seed, w.batch, w.L, w.D, w.N, w.io)
     p = I.make_params(w.seed, w.D, w.N)
-    g = {k: up(v) for k, v in s.items()}
-    A, Dk = up(p["A"]), up(p["Dskip"])
-    dy = up(I.f32_to_bf16_bits(I.make_state(w.seed + 9, w.batch, w.L, w.D)))
+    g = {k: _up(v, dev) for k, v in s.items()}
+    A, Dk = _up(p["A"], dev), _up(p["Dskip"], dev)
+    dy = _up(I.f32_to_bf16_bits(I.make_state(w.seed + 9, w.batch, w.L, w.D)), dev)
     y = torch.empty((w.batch, w.L, w.D), dtype=torch.bfloat16, device=dev)
     bnd = torch.empty((w.batch, w.L // w.K, w.D, w.N), dtype=torch.float32, device=dev)
     ws = torch.empty(bdscan.train_blocks_backward_workspace_bytes(g["x"], g["B"], w.K), dtype=torch.uint8,
@@ -695,39 +774,29 @@ def run_train_step(args):
     def bwd():
         bdscan.train_blocks_backward(g["x"], g["dt"], A, g["B"], g["C"], Dk, w.K, dy, bnd, grads=grads, ws=ws)
 
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(warmup):
         fwd()
         bwd()
     torch.cuda.synchronize(dev)
-    n = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
-    with ClockSampler(0) as clk:
-        for i in range(n):
-            evs[i][0].record()
-            fwd()
-            evs[i][1].record()
-            bwd()
-            evs[i][2].record()
-        torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        evs[i][0].record()
+        fwd()
+        evs[i][1].record()
+        bwd()
+        evs[i][2].record()
+    torch.cuda.synchronize(dev)
     f_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     b_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    tok = w.batch * w.L
-    ex2_peak = EX2_PER_CLK_SM * SM_COUNT * peaks["sm_max_mhz"] * 1e-3
     elem = w.batch * w.L * w.D * w.N
-    line = {"metric": METRIC, "workload": "train_fwd_bwd", "n_gpus": 1, "steps": n, "dtype": "f32",
-            "data": "synthetic",
-            "config": {"batch": w.batch, "seq_len": w.L, "d_inner": w.D, "d_state": w.N, "block": w.K,
+    return {"config": {"batch": w.batch, "seq_len": w.L, "d_inner": w.D, "d_state": w.N, "block": w.K,
                        "io_dtype": w.io, "gated": False},
             "forward_ms": f_ms, "backward_ms": b_ms, "step_ms": f_ms + b_ms,
-            "tokens_per_s": tok / ((f_ms + b_ms) * 1e-3),
-            "backward": {"kernels": 2, "ex2_frac": elem / (b_ms * 1e-3) / 1e9 / ex2_peak,
+            "tokens_per_s": w.batch * w.L / ((f_ms + b_ms) * 1e-3),
+            "backward": {"kernels": 2, "sfu_frac": elem / (b_ms * 1e-3) / 1e9 / ex2_peak_g(peaks),
                          "hbm_gbs": backward_bytes(w) / (b_ms * 1e-3) / 1e9,
                          "hbm_frac": backward_bytes(w) / (b_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                         "algorithmic_bytes": backward_bytes(w),
-                         "workspace_bytes": ws.numel()},
-            "gpu_launches": 3 * n, "clocks": clk.summary()}
-    print(json.dumps(line), flush=True)
-    return 0
+                         "algorithmic_bytes": backward_bytes(w), "workspace_bytes": ws.numel()}}
 
 
 def run_context_parallel(args):
@@ -800,6 +869,82 @@ def run_context_parallel(args):
     return 0
 
 
+PROFILE_CASES = {
+    # name: (workload the case reduces, batch, L, D, N, K, op)
+    "stack_k4": ("stack350m", 4, 8192, 2048, 64, 4, "train"),
+    "stack_k16": ("stack350m", 4, 8192, 2048, 64, 16, "train"),
+    "stack_k64": ("stack350m", 4, 8192, 2048, 64, 64, "train"),
+    "train_k16": ("train", 8, 4096, 1536, 16, 16, "train_states"),
+    "backward_k16": ("train", 8, 4096, 1536, 16, 16, "backward"),
+    "prefill262k_rows": ("step262k", 4, 32768, 2048, 16, 32, "prefill"),
+    "prefill65k_chunked": ("step65k", 1, 65536, 1536, 16, 32, "prefill_chunked"),
+    "step65k": ("step65k", 1, 32, 1536, 16, 32, "step"),
+    "step262k": ("step262k", 4, 32, 2048, 16, 32, "step"),
+}
+
+
+def run_profile_case(name, warm=3, reps=5):
+    """One kernel case, reduced from a workload to a size an ncu capture
+    finishes quickly (inputs still larger than L2 where the workload's are):
+    `warm` untimed calls, then `reps` timed ones. The stack cases keep the
+    stack's grid shape per wave at a quarter of its batch, the 262K prefill
+    case keeps its 256 CTAs at an eighth of the context."""
+    import torch
+    from selective_ssm_scan_mamba_b200 import bdscan
+    wname, Bt, L, D, N, K, op = PROFILE_CASES[name]
+    w = I.WORKLOADS[wname]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    s = I.make_sequence(w.seed, Bt, L, D, N, w.io)
+    p = I.make_params(w.seed, D, N)
+    g = {k: _up(v, dev) for k, v in s.items()}
+    A, Dk = _up(p["A"], dev), _up(p["Dskip"], dev)
+    y = torch.empty((Bt, L, D), dtype=torch.bfloat16, device=dev)
+    if op == "train":
+        fn = lambda: bdscan.train_blocks(g["x"], g["dt"], A, g["B"], g["C"], Dk, K, y=y)  # noqa: E731
+    elif op in ("train_states", "backward"):
+        bnd = torch.empty((Bt, L // K, D, N), dtype=torch.float32, device=dev)
+        ho = torch.empty((Bt, D, N), dtype=torch.float32, device=dev)
+        fn = lambda: bdscan.train_blocks(g["x"], g["dt"], A, g["B"], g["C"], Dk, K, y=y, boundary=bnd,  # noqa: E731
+                                         h_out=ho)
+        if op == "backward":
+            fn()
+            dy = _up(I.f32_to_bf16_bits(I.make_state(w.seed + 9, Bt, L, D)), dev)
+            ws = torch.empty(bdscan.train_blocks_backward_workspace_bytes(g["x"], g["B"], K), dtype=torch.uint8,
+                             device=dev)
+            gr = {}
+            fn = lambda: bdscan.train_blocks_backward(g["x"], g["dt"], A, g["B"], g["C"], Dk, K, dy, bnd,  # noqa
+                                                      ws=ws, grads=gr)
+    elif op == "prefill":
+        ho = torch.empty((Bt, D, N), dtype=torch.float32, device=dev)
+        fn = lambda: bdscan.prefill(g["x"], g["dt"], A, g["B"], g["C"], Dk, K, y=y, h_out=ho)  # noqa: E731
+    elif op == "prefill_chunked":
+        ho = torch.empty((Bt, D, N), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(16, bdscan.prefill_chunked_workspace_bytes(g["x"], g["B"], K)), dtype=torch.uint8,
+                         device=dev)
+        fn = lambda: bdscan.prefill_chunked(g["x"], g["dt"], A, g["B"], g["C"], Dk, K, y=y, h_out=ho,  # noqa
+                                            ws=ws)
+    else:   # one block step from a random cache
+        hc = _up(I.make_state(w.seed + 5, Bt, D, N, scale=0.5), dev)
+        fn = lambda: bdscan.block_step(g["x"], g["dt"], A, g["B"], g["C"], Dk, hc, y=y)  # noqa: E731
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize(dev)
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ts.append(e0.elapsed_time(e1))
+    ms = statistics.median(ts)
+    elem = Bt * L * D * N
+    print(json.dumps({"profile_case": name, "batch": Bt, "L": L, "D": D, "N": N, "K": K, "op": op, "ms": ms,
+                      "sfu_frac": elem / (ms * 1e-3) / 1e9 / ex2_peak_g(load_peaks())}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -808,21 +953,33 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
-    ap.add_argument("--workload", default="train",
-                    choices=["train", "train_fwd_bwd", "step65k", "step262k", "stack350m", "cp_prefill"],
-                    help="train: the headline line; the others print their own measurement lines")
+    ap.add_argument("--no-secondary", action="store_true", help="headline only (profiling runs)")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+                    help="run one reduced kernel case (for ncu captures) and exit")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=[WORKLOAD, "train", "train_fwd_bwd", "step65k", "step262k", "cp_prefill"],
+                    help=f"{WORKLOAD}: the headline line; the others print one measurement line each")
     args = ap.parse_args()
-    if args.workload in ("step65k", "step262k"):
-        return run_inference(args, args.workload)
-    if args.workload == "stack350m":
-        return run_stack(args)
-    if args.workload == "train_fwd_bwd":
-        return run_train_step(args)
+    if args.profile_case:
+        return run_profile_case(args.profile_case, max(args.warmup, 1), max(args.steps, 1))
     if args.workload == "cp_prefill":
         return run_context_parallel(args)
     if args.impl == "reference":
         return run_reference(args)
-    return run_ours(args)
+    if args.workload == WORKLOAD:
+        return run_ours(args)
+    import torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    if args.workload == "train":
+        rec = measure_train(dev, peaks, args.steps, max(args.warmup, 3))
+    elif args.workload == "train_fwd_bwd":
+        rec = measure_train_step(dev, peaks, args.steps, max(args.warmup, 3))
+    else:
+        rec = measure_inference(args.workload, dev, peaks)
+    print(json.dumps({"metric": METRIC, "workload": args.workload, "n_gpus": 1, **rec}), flush=True)
+    return 0
 
 
 if __name__ == "__main__":

@@ -26,3 +26,17 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Worst state errors of the run, normwise (asserted) and per element (reported)."""
+    mod = sys.modules.get("tests.gpu_util")
+    log = getattr(mod, "STATE_LOG", None) if mod else None
+    if not log:
+        return
+    tr = terminalreporter
+    tr.section("state checks: normwise (asserted) and per-element ratio (reported)")
+    tr.write_line(f"{len(log)} checks; worst normwise {max(r[1] for r in log):.3g} of tolerance, "
+                  f"worst per-element {max(r[2] for r in log):.3g} of tolerance")
+    for what, nw, pe in sorted(log, key=lambda r: -r[2])[:8]:
+        tr.write_line(f"  {what}: normwise {nw:.3g}, per-element {pe:.3g}")

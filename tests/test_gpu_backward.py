@@ -86,10 +86,13 @@ def test_backward_vs_oracle(bd, Bt, L, D, N, K, io, gated, with_h0, sp):
 
 
 def test_backward_at_training_size_sampled(bd):
-    """Batch 8 x 4096 tokens x 1536 channels, N = 16, blocks of 16, bf16: the
-    oracle recomputes a sample of channels in full (channels are independent
-    for dx, d(dt), dz, dA, dDskip); dB and dC are checked through the
-    homogeneity identity sum(C dC) + sum(Dskip dDskip) = sum(dy y)."""
+    """Batch 8 x 4096 tokens x 1536 channels, N = 16, blocks of 16, bf16.
+    dx and d(dt) depend only on their own channel, dA and dDskip on their
+    channel summed over the batch: the oracle recomputes a sample of channels
+    in full for those. dB[b] and dC[b] sum over all channels of batch row b
+    only (the GPU reduces 48 CTA partial rows per token): the oracle runs
+    batch row 0 in full (4096 x 1536) and they are checked element by
+    element there, together with that row's dx and d(dt)."""
     Bt, L, D, N, K = 8, 4096, 1536, 16, 16
     s = I.make_sequence(1, Bt, L, D, N, "bf16")
     s.update(I.make_params(1, D, N))
@@ -108,12 +111,12 @@ def test_backward_at_training_size_sampled(bd):
         assert_c12(to_f64(out[k])[:, :, ch], want[k], RTOL_GRAD["bf16"], k)
     assert_state(to_f64(out["dA"])[ch][None], want["dA"][None], "dA", rtol=RTOL_GRAD["param"])
     assert_c12(to_f64(out["dDskip"])[ch], want["dDskip"], RTOL_GRAD["param"], "dDskip")
-    # Euler identity in (C, Dskip): y is linear in them jointly
-    yf = to_f64(y)
-    dyf = oracle.decode(dy)
-    lhs = float(np.sum(oracle.decode(s["C"]) * to_f64(out["dC"])) + np.sum(s["Dskip"].astype(np.float64) * to_f64(out["dDskip"])))
-    rhs = float(np.sum(dyf * yf))
-    assert abs(lhs - rhs) <= 2e-2 * (np.sqrt(np.sum(dyf * dyf) * np.sum(yf * yf)) / np.sqrt(yf.size)) * 10 + 1e-3 * abs(rhs)
+    # batch row 0 in full: dB and dC element by element
+    row = {k: np.ascontiguousarray(s[k][:1]) for k in ("x", "dt", "B", "C")}
+    want0 = oracle.train_blocks_backward(row["x"], row["dt"], s["A"], row["B"], row["C"], s["Dskip"], K,
+                                         np.ascontiguousarray(dy[:1]))
+    for k in ("dB", "dC", "dx", "ddt"):
+        assert_c12(to_f64(out[k])[:1], want0[k], RTOL_GRAD["bf16"], f"{k} (batch row 0)")
 
 
 def test_backward_is_deterministic(bd):

@@ -1,14 +1,16 @@
 """The allocation-free time-chunked prefill (bdscan_prefill_chunked_noalloc),
 called through the C ABI, against the entry point that takes a caller
-workspace (bdscan_prefill_chunked). Two calls in a row share the library's
-fixed device scratch, so the second one also shows that nothing left there by
-the first leaks into its result."""
+workspace (bdscan_prefill_chunked). Both run the same kernels on the same
+inputs, so their outputs must be bit-identical. The allocation-free calls run
+back to back and share the library's fixed device scratch: the third call has
+the first call's shape (another seed), so anything stale the earlier calls
+left in the scratch would sit exactly where it reads."""
 import ctypes as ct
 
 import pytest
 
 from selective_ssm_scan_mamba_b200 import inputs as I
-from tests.gpu_util import RTOL_Y, assert_c12, assert_state, to_dev, to_f64
+from tests.gpu_util import to_dev
 
 SCRATCH_BYTES = 8 << 20   # the fixed scratch the header states
 
@@ -18,10 +20,15 @@ def _abi():
     return bdscan
 
 
+def s_seed(s):
+    return s["seed"]
+
+
 def _case(seed, Bt, L, D, N, io, gated, with_h0):
     s = I.make_sequence(seed, Bt, L, D, N, io, gated=gated)
     s.update(I.make_params(seed, D, N))
     s["h0"] = I.make_state(seed + 1, Bt, D, N, scale=0.5) if with_h0 else None
+    s["seed"] = seed
     return s
 
 
@@ -32,15 +39,17 @@ def _dims_inputs(bd, g, Bt, L, D, N, K, io):
     return dims, ins
 
 
-# (seed, Bt, L, D, N, K, io, gated, h0): both take the chunked path with under 8 MiB of scratch
+# (seed, Bt, L, D, N, K, io, gated, h0): all take the chunked path with under
+# 8 MiB of scratch; the third repeats the first one's shape with new inputs
 CASES = [
     (501, 1, 8192, 512, 16, 16, "bf16", True, True),
     (502, 2, 2048, 64, 64, 32, "f32", False, True),
+    (503, 1, 8192, 512, 16, 16, "bf16", True, False),
 ]
 
 
 @pytest.mark.gpu
-def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
+def test_noalloc_matches_workspace_entry_point_on_calls_in_a_row():
     import torch
     bd = _abi()
     lib = bd.raw_library()
@@ -48,7 +57,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
     runs = []
     for seed, Bt, L, D, N, K, io, gated, with_h0 in CASES:
         s = _case(seed, Bt, L, D, N, io, gated, with_h0)
-        g = {k: (None if v is None else to_dev(v)) for k, v in s.items()}
+        g = {k: (None if v is None else to_dev(v)) for k, v in s.items() if k != "seed"}
         dims, ins = _dims_inputs(bd, g, Bt, L, D, N, K, io)
         need = int(lib.bdscan_prefill_chunked_workspace(ct.byref(dims)))
         assert 0 < need <= SCRATCH_BYTES, need
@@ -57,7 +66,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
                    h=torch.empty((Bt, D, N), device="cuda"),
                    b=torch.empty((Bt, L // K, D, N), device="cuda"))
         runs.append((s, g, dims, ins, need, out, K, io))
-    # the two allocation-free calls, back to back on one stream
+    # the allocation-free calls, back to back on one stream
     for s, g, dims, ins, need, out, K, io in runs:
         h0 = None if g["h0"] is None else g["h0"].data_ptr()
         rc = lib.bdscan_prefill_chunked_noalloc(ct.byref(dims), ct.byref(ins), h0, out["y"].data_ptr(),
@@ -73,9 +82,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
                                         ref["b"].data_ptr(), ws.data_ptr(), need, stream)
         assert rc == 0, lib.bdscan_status_string(rc).decode()
         torch.cuda.synchronize()
-        assert_c12(to_f64(out["y"]), to_f64(ref["y"]), RTOL_Y[io], "y")
-        assert_state(to_f64(out["h"]), to_f64(ref["h"]), "final state")
-        assert_state(to_f64(out["b"]), to_f64(ref["b"]), "boundary states")
+        for k in ("y", "h", "b"):
+            assert torch.equal(out[k], ref[k]), f"seed {s_seed(s)}: {k} differs from the workspace entry point"
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
