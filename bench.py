@@ -187,9 +187,10 @@ def _oracle_worker(conn):
     import oracle
     oracle.load()
     job = conn.recv()
+    fn = oracle.prefill if job.get("op") == "prefill" else oracle.train_blocks
     conn.send("ready")
     while conn.recv() == "run":
-        oracle.train_blocks(job["x"], job["dt"], job["A"], job["B"], job["C"], job["Dskip"], job["K"])
+        fn(job["x"], job["dt"], job["A"], job["B"], job["C"], job["Dskip"], job["K"])
         conn.send("done")
 
 
@@ -211,7 +212,7 @@ class OraclePool:
     the wall-clock time until the last is done. s: x, dt [n_seq, L, channels],
     B, C [n_seq, L, N]; A [channels, N], Dskip [channels]."""
 
-    def __init__(self, s, A, Dskip, K, workers=None):
+    def __init__(self, s, A, Dskip, K, workers=None, op="train"):
         import multiprocessing as mp
         nch = s["x"].shape[2]
         self.workers = max(1, min(workers or os.cpu_count() or 1, nch))
@@ -224,7 +225,7 @@ class OraclePool:
             pr.start()
             a.send({"x": np.ascontiguousarray(s["x"][:, :, c0:c1]), "dt": np.ascontiguousarray(s["dt"][:, :, c0:c1]),
                     "B": s["B"], "C": s["C"], "A": np.ascontiguousarray(A[c0:c1]),
-                    "Dskip": np.ascontiguousarray(Dskip[c0:c1]), "K": K})
+                    "Dskip": np.ascontiguousarray(Dskip[c0:c1]), "K": K, "op": op})
             self.conns.append(a)
             self.procs.append(pr)
         for c in self.conns:
@@ -650,7 +651,18 @@ def measure_inference(name, dev, peaks) -> dict:
     host_us = (time.perf_counter() - t0) / len(qs) * 1e6
     torch.cuda.synchronize(dev)
     eager_us = (time.perf_counter() - t0) / len(qs) * 1e6
-    del qs
+    # the same through a prepared bdscan.BlockStep (A, Dskip, cache checked once)
+    prep = bdscan.BlockStep(A, Dk, cache, K)
+    for q in qs[:10]:
+        prep(q["x"], q["dt"], q["B"], q["C"], y=y_step)
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    for q in qs:
+        prep(q["x"], q["dt"], q["B"], q["C"], y=y_step)
+    prep_host_us = (time.perf_counter() - t0) / len(qs) * 1e6
+    torch.cuda.synchronize(dev)
+    prep_us = (time.perf_counter() - t0) / len(qs) * 1e6
+    del qs, prep
 
     # the whole denoise loop (all blocks: steps + commit) as one CUDA graph
     cache0 = cache.clone()
@@ -723,6 +735,7 @@ def measure_inference(name, dev, peaks) -> dict:
                  "hbm_frac": per / (step_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
                  "sfu_frac": w.batch * K * w.D * w.N / (step_us * 1e-6) / 1e9 / sfu,
                  "eager_call_us": eager_us, "eager_host_us": host_us,
+                 "prepared_call_us": prep_us, "prepared_host_us": prep_host_us,
                  "inputs": f"rotating pool of {pool_n} step inputs ({pool_n * per / 1e6:.0f} MB > 2x L2)"},
         "loop": {"ms": loop_ms, "graph_launches": launches, "us_per_launch": loop_ms * 1e3 / launches,
                  "committed_tokens_per_s": w.batch * K * w.blocks / (loop_ms * 1e-3),
@@ -869,6 +882,88 @@ def run_context_parallel(args):
     return 0
 
 
+def _oracle_sample(name):
+    """Bounded oracle sample of a workload's timed unit: (inputs, params, what the
+    unit is, element-steps of the full unit / of the sample, call). Channels are
+    independent, so the cost of the unit is exactly linear in the channels and
+    sequences sampled; config 5 also multiplies by its 24 layers."""
+    import oracle
+    w = I.WORKLOADS[name]
+    if name == "pr1":
+        chans, n_seq, L, op, unit = list(range(w.D)), w.batch, w.L, "train", "train_blocks, 256 tokens"
+    elif name == "train":
+        chans, n_seq, L, op, unit = list(range(192)), w.batch, w.L, "train", "train_blocks, 8 x 4096 tokens"
+    elif name == "stack350m":
+        chans, n_seq, L, op, unit = list(range(32)), w.batch, w.L, "train", "24 layers, 16 x 8192 tokens, K = 16"
+    else:   # inference: the context prefill (forward-only scan) of all sequences
+        chans, n_seq, L, op, unit = list(range(64)), w.batch, 8192, "prefill", \
+            f"prefill of {w.batch} x {w.L} context tokens"
+    s = I.make_sequence(w.seed, n_seq, L, w.D, w.N, w.io, stream="seq" if op == "train" else ("context",),
+                        channels=chans)
+    p = I.make_params(w.seed, w.D, w.N)
+    A, Dk = p["A"][chans], p["Dskip"][chans]
+    full = w.batch * w.L * w.D * w.N * w.layers
+    part = n_seq * L * len(chans) * w.N
+    if op == "train":
+        fn = lambda: oracle.train_blocks(s["x"], s["dt"], A, s["B"], s["C"], Dk, w.K)  # noqa: E731
+    else:
+        fn = lambda: oracle.prefill(s["x"], s["dt"], A, s["B"], s["C"], Dk, w.K)  # noqa: E731
+    return s, A, Dk, unit, full, part, fn, op
+
+
+def baseline_table(bench_path=None) -> str:
+    """Markdown rows of the oracle (single thread and all host cores) and of the
+    GPU (from a bench.py JSON line) per workload."""
+    import oracle
+    oracle.load()
+    gpu = json.load(open(bench_path)) if bench_path else {}
+    sec = gpu.get("secondary", {})
+    rows = ["| config | timed unit | oracle 1 thread | oracle all cores | GPU (this build) | GPU tokens/s | "
+            "HBM GB/s (% of measured / of 8000) | SFU % |", "|---|---|---|---|---|---|---|---|"]
+    for cfg, name in enumerate(["pr1", "train", "step65k", "step262k", "stack350m"], start=1):
+        w = I.WORKLOADS[name]
+        s, A, Dk, unit, full, part, fn, op = _oracle_sample(name)
+        t0 = time.perf_counter()
+        fn()
+        t1 = (time.perf_counter() - t0) * full / part
+        pool = OraclePool(s, A, Dk, w.K, op=op)
+        try:
+            ta = pool.step() * full / part
+        finally:
+            pool.close()
+        gcol = tcol = hcol = scol = "-"
+        if name == "stack350m" and gpu.get("value"):
+            gcol = f"{gpu['ms_per_step']:.1f} ms per step"
+            tcol = f"{gpu['value'] / 1e6:.1f} M"
+            hb = gpu["roofline"]["hbm"]
+            hcol = f"{hb['achieved']:.0f} ({100 * hb['frac']:.1f} % / {100 * hb['frac_of_nominal_8000']:.1f} %)"
+            scol = f"{100 * gpu['roofline']['frac']:.1f}"
+        elif name == "train" and "train" in sec and "ms" in sec["train"]:
+            r = sec["train"]
+            gcol, tcol = f"{r['ms']:.3f} ms", f"{r['tokens_per_s'] / 1e6:.1f} M"
+            hb = r["roofline"]["hbm"]
+            hcol = f"{hb['achieved']:.0f} ({100 * hb['frac']:.1f} % / {100 * hb['frac_of_nominal_8000']:.1f} %)"
+            scol = f"{100 * r['roofline']['frac']:.1f}"
+        elif name in sec and "prefill" in sec[name]:
+            r = sec[name]["prefill"]
+            gcol, tcol = f"{r['ms']:.2f} ms", f"{r['tokens_per_s'] / 1e6:.1f} M"
+            hcol = f"{r['hbm_gbs']:.0f} ({100 * r['hbm_frac']:.1f} % / {100 * r['hbm_gbs'] / 8000:.1f} %)"
+            scol = f"{100 * r['sfu_frac']:.1f}"
+        tokens = w.batch * w.L * w.layers
+
+        def sec_(v):
+            return f"{v * 1e3:.1f} ms" if v < 1 else f"{v:.1f} s"
+        label = f"{cfg} {name}"
+        rows.append(f"| {label} | {unit} | {sec_(t1)} ({tokens / t1 / 1e3:.1f} K tok/s) | {sec_(ta)} "
+                    f"({tokens / ta / 1e3:.1f} K tok/s, {pool.workers} cores) | {gcol} | {tcol} | {hcol} | {scol} |")
+    rows.append("")
+    rows.append(f"Oracle: `oracle/bdscan_oracle.c` (fp64, single-threaded C) on {cpu_model() or 'the host'}; "
+                "all-cores = one spawned process per core over channel slices. Timed on bounded channel samples "
+                "and extrapolated linearly (the cost is exactly linear in channels, sequences and layers); the "
+                "inference rows time the forward-only prefill of the context.")
+    return "\n".join(rows)
+
+
 PROFILE_CASES = {
     # name: (workload the case reduces, batch, L, D, N, K, op)
     "stack_k4": ("stack350m", 4, 8192, 2048, 64, 4, "train"),
@@ -954,12 +1049,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--no-secondary", action="store_true", help="headline only (profiling runs)")
+    ap.add_argument("--baseline-table", nargs="?", const="", metavar="BENCH_JSON",
+                    help="print the oracle / GPU table of every workload (GPU columns from a bench.py JSON line)")
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
                     help="run one reduced kernel case (for ncu captures) and exit")
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=[WORKLOAD, "train", "train_fwd_bwd", "step65k", "step262k", "cp_prefill"],
                     help=f"{WORKLOAD}: the headline line; the others print one measurement line each")
     args = ap.parse_args()
+    if args.baseline_table is not None:
+        print(baseline_table(args.baseline_table or None))
+        return 0
     if args.profile_case:
         return run_profile_case(args.profile_case, max(args.warmup, 1), max(args.steps, 1))
     if args.workload == "cp_prefill":

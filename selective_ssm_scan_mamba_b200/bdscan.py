@@ -83,6 +83,10 @@ def _ptr(t):
 
 
 def _need(t, name, dtype, shape, device):
+    # one combined test on the common path; the specific error only on failure
+    if (isinstance(t, torch.Tensor) and t.dtype == dtype and t.shape == shape and t.is_contiguous()
+            and t.device == device):
+        return
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.device != device:
@@ -123,7 +127,13 @@ def _check_device(device):
         raise ValueError("bdscan runs on CUDA tensors only")
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(dev):
+    """The current CUDA stream of dev as a raw handle (the call is queued there)."""
+    if _raw_stream is not None:
+        return _raw_stream(dev.index if dev.index is not None else torch.cuda.current_device())
     return torch.cuda.current_stream(dev).cuda_stream
 
 
@@ -315,6 +325,55 @@ def block_step(x, dt, A, B, C, Dskip, h_cache, z=None, dt_softplus=True, y=None)
     rc = _lib.bdscan_block_step(ct.byref(dims), ct.byref(ins), _ptr(h_cache), _ptr(y), _stream(dev))
     _check(rc, "bdscan_block_step")
     return y
+
+
+class BlockStep:
+    """A block step prepared for one shape, for denoising loops that call it
+    many times: A, Dskip and the cache are checked once here, and each call
+    checks only the step's own tensors (shape, dtype, device, contiguity) and
+    marshals pointers. Calling it returns y = bdscan_block_step(x, dt, B, C)
+    with the prepared A, Dskip, h_cache (read only) and gate flag; y may be
+    passed in to avoid an allocation."""
+
+    def __init__(self, A, Dskip, h_cache, block, dtype=torch.bfloat16, dt_softplus=True, gated=False):
+        if not isinstance(h_cache, torch.Tensor) or h_cache.dim() != 3:
+            raise ValueError("h_cache must be a [batch, D, N] tensor")
+        _check_device(h_cache.device)
+        Bt, D, N = h_cache.shape
+        dev = h_cache.device
+        if dtype not in (torch.float32, torch.bfloat16):
+            raise TypeError("io dtype must be float32 or bfloat16")
+        _need(h_cache, "h_cache", torch.float32, (Bt, D, N), dev)
+        _need(A, "A", torch.float32, (D, N), dev)
+        _need(Dskip, "Dskip", torch.float32, (D,), dev)
+        self._keep = (A, Dskip, h_cache)   # the prepared pointers stay valid while this object lives
+        self.dev, self.io, self.gated = dev, dtype, bool(gated)
+        K = int(block)
+        self.xshape, self.bshape = torch.Size((Bt, K, D)), torch.Size((Bt, K, N))
+        self._dims = Dims(Bt, K, D, N, K, BF16 if dtype == torch.bfloat16 else F32, 1 if dt_softplus else 0)
+        self._ins = Inputs(None, None, None, None, None, A.data_ptr(), Dskip.data_ptr())
+        self._h = h_cache.data_ptr()
+        self._dims_ref, self._ins_ref = ct.byref(self._dims), ct.byref(self._ins)
+
+    def __call__(self, x, dt, B, C, y=None, z=None):
+        xs, bs, io, dev = self.xshape, self.bshape, self.io, self.dev
+        for t, name, shp in ((x, "x", xs), (dt, "dt", xs), (B, "B", bs), (C, "C", bs)):
+            _need(t, name, io, shp, dev)
+        if self.gated:
+            _need(z, "z", io, xs, dev)
+        elif z is not None:
+            raise ValueError("this BlockStep was prepared without a gate")
+        if y is None:
+            y = torch.empty(xs, dtype=io, device=dev)
+        else:
+            _need(y, "y", io, xs, dev)
+        ins = self._ins
+        ins.x, ins.dt, ins.B, ins.C = x.data_ptr(), dt.data_ptr(), B.data_ptr(), C.data_ptr()
+        ins.z = z.data_ptr() if self.gated else None
+        rc = _lib.bdscan_block_step(self._dims_ref, self._ins_ref, self._h, y.data_ptr(), _stream(dev))
+        if rc != 0:
+            raise BdscanError(rc, "bdscan_block_step")
+        return y
 
 
 def commit_block(x, dt, A, B, C, Dskip, h_cache, z=None, dt_softplus=True, want_y=False, y=None):

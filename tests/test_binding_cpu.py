@@ -127,3 +127,34 @@ def test_noalloc_prefill_needs_caller_outputs(fake):
     assert args[3] == y.data_ptr() and args[4] == h.data_ptr() and args[5] is None and args[6] == 1234
     with pytest.raises(ValueError):   # outputs are checked like inputs
         bdscan.prefill_chunked_noalloc(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], 16, y[:, :16], h)
+
+
+def test_prepared_block_step_marshalling(fake):
+    t = tensors(L=32)
+    h = torch.zeros(2, 64, 16)
+    step = bdscan.BlockStep(t["A"], t["Dskip"], h, 32)
+    y = step(t["x"], t["dt"], t["B"], t["C"])
+    name, args = fake.calls[-1]
+    assert name == "bdscan_block_step"
+    d = _dims(args[0]._obj)
+    assert (d.batch, d.seqlen, d.d_inner, d.d_state, d.block, d.io_dtype, d.dt_softplus) == (2, 32, 64, 16, 32, 1, 1)
+    ins = args[1]._obj
+    assert (ins.x, ins.dt, ins.B, ins.C, ins.z) == (t["x"].data_ptr(), t["dt"].data_ptr(), t["B"].data_ptr(),
+                                                    t["C"].data_ptr(), None)
+    assert (ins.A, ins.Dskip) == (t["A"].data_ptr(), t["Dskip"].data_ptr())
+    assert args[2] == h.data_ptr() and args[3] == y.data_ptr() and args[4] == 1234
+    y2 = torch.empty_like(y)
+    assert step(t["x"], t["dt"], t["B"], t["C"], y=y2) is y2
+    with pytest.raises(ValueError, match="shape"):        # a block of another length
+        step(t["x"][:, :16].contiguous(), t["dt"], t["B"], t["C"])
+    with pytest.raises(TypeError, match="dtype"):
+        step(t["x"].float(), t["dt"], t["B"], t["C"])
+    with pytest.raises(ValueError, match="gate"):
+        step(t["x"], t["dt"], t["B"], t["C"], z=t["x"])
+    with pytest.raises(ValueError, match="shape"):        # A of another width than the cache
+        bdscan.BlockStep(torch.zeros(32, 16), t["Dskip"], h, 32)
+    gated = bdscan.BlockStep(t["A"], t["Dskip"], h, 32, gated=True)
+    with pytest.raises(TypeError, match="Tensor"):
+        gated(t["x"], t["dt"], t["B"], t["C"])
+    gated(t["x"], t["dt"], t["B"], t["C"], z=t["x"])
+    assert fake.calls[-1][1][1]._obj.z == t["x"].data_ptr()
