@@ -103,8 +103,8 @@ typedef struct {
  * Optional outputs: boundary states after each block (NULL = not written) and
  * the final state h_out (NULL = not written). Blocks longer than 32 tokens
  * first sweep the reverse state alone and keep its value at every 16-token
- * span start in shared memory ((ceil(K/16) - 1) x N x 128 bytes: K up to 1392
- * at N = 16 and 304 at N = 64 with bf16 I/O, 1200 and 240 with fp32), then run
+ * span start in shared memory ((ceil(K/16) - 1) x N x 128 bytes: K up to 1408
+ * at N = 16 and 320 at N = 64 with bf16 I/O, 1216 and 256 with fp32), then run
  * the fused pass span by span. Where that does not fit, a two-sweep path stages
  * the block's reverse readout in shared memory instead (K <= 768); blocks too
  * long for both return BDSCAN_ERR_UNSUPPORTED.
@@ -135,7 +135,8 @@ int bdscan_prefill(const bdscan_dims *dims, const bdscan_inputs *in,
  * rounding, not bit for bit (use bdscan_prefill where the cache must equal a
  * commit chain exactly). Two exps per (token, channel, state). When a single
  * chunk already fills the device the call runs bdscan_prefill's sequential
- * scan instead (workspace size 0).
+ * scan instead (workspace size 0). The number of chunks keeps all CTAs of a
+ * pass resident at once (rows x chunks <= SMs x resident CTAs per SM).
  * ws: device scratch of bdscan_prefill_chunked_workspace(dims) bytes (the
  * size depends on the current device's SM count), 16-byte aligned, owned by
  * the caller, not preserved; BDSCAN_ERR_WORKSPACE if it is missing or too
@@ -152,7 +153,9 @@ int bdscan_prefill_chunked(const bdscan_dims *dims, const bdscan_inputs *in, con
  * Scratch is a fixed 8 MiB array in device memory that the library holds on
  * every GPU it is loaded on until the process exits; problems whose
  * bdscan_prefill_chunked_workspace(dims) exceeds 8 MiB return
- * BDSCAN_ERR_WORKSPACE (use bdscan_prefill_chunked with your own buffer).
+ * BDSCAN_ERR_WORKSPACE (use bdscan_prefill_chunked with your own buffer);
+ * the chunk plan keeps its CTAs to one wave, so on a 148-SM B200 no size
+ * needs more than about 2.5 MB.
  * The first call on a device looks up the array's device address (a CUDA
  * runtime query, done once per device); make that first call before any
  * stream capture. The address is kept for the life of the process, so the

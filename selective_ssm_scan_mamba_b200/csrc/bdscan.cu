@@ -54,8 +54,11 @@ bool long_fused_fits(int64_t K) {
     return bdk::Layout<IO, N, bdk::kLongFused, 0>::base_bytes + long_fused_ck_bytes(K, N) <= (size_t)kMaxDynSmem;
 }
 
+// pdl: launch with programmatic stream serialisation, so that the kernel's
+// launch overlaps the end of the previous kernel in the stream (the kernel
+// waits for it before touching global memory).
 template <class IO, int N, int MODE, int KC, int NPTV = 4>
-int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1) {
+int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1, bool pdl = false) {
     using CF = bdk::Cfg<N, MODE, KC, NPTV>;
     using LY = bdk::Layout<IO, N, MODE, KC, NPTV>;
     const size_t smem = LY::base_bytes + (MODE == bdk::kLong ? (size_t)a.K * bdk::kCh * 4
@@ -74,7 +77,22 @@ int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz =
         done_mask.fetch_or(bit, std::memory_order_acq_rel);
     }
     dim3 grid((unsigned)((a.D + bdk::kCh - 1) / bdk::kCh), (unsigned)batch, gz);
-    kern<<<grid, CF::THREADS, smem, st>>>(a);
+    if (pdl) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(CF::THREADS);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, a);
+        if (le != cudaSuccess) { (void)cudaGetLastError(); g_last_cuda = le; return BDSCAN_ERR_CUDA; }
+    } else {
+        kern<<<grid, CF::THREADS, smem, st>>>(a);
+    }
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
     return BDSCAN_OK;
@@ -82,26 +100,32 @@ int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz =
 
 template <class IO, int N>
 int dispatch_mode(int mode, const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1,
-                  bool thin = false) {
+                  bool thin = false, bool pdl = false) {
     if constexpr (N == 16) {
         if (thin && mode == bdk::kFused) {   // one state per lane: the latency-bound small block step
             switch (a.K) {
-                case 4: return launch<IO, N, bdk::kFused, 4, 1>(a, batch, st);
-                case 16: return launch<IO, N, bdk::kFused, 16, 1>(a, batch, st);
-                case 32: return launch<IO, N, bdk::kFused, 32, 1>(a, batch, st);
-                default: return launch<IO, N, bdk::kFused, 0, 1>(a, batch, st);
+                case 4: return launch<IO, N, bdk::kFused, 4, 1>(a, batch, st, 1, pdl);
+                case 16: return launch<IO, N, bdk::kFused, 16, 1>(a, batch, st, 1, pdl);
+                case 32: return launch<IO, N, bdk::kFused, 32, 1>(a, batch, st, 1, pdl);
+                default: return launch<IO, N, bdk::kFused, 0, 1>(a, batch, st, 1, pdl);
             }
         }
     }
-    if (mode == bdk::kForwardOnly) return launch<IO, N, bdk::kForwardOnly, 0>(a, batch, st, gz);
-    if (mode == bdk::kLong) return launch<IO, N, bdk::kLong, 0>(a, batch, st);
-    if (mode == bdk::kLongFused) return launch<IO, N, bdk::kLongFused, 0>(a, batch, st);
-    if (mode == bdk::kReverseAcc) return launch<IO, N, bdk::kReverseAcc, 0>(a, batch, st);
+    if constexpr (N == 64) {
+        if (mode == bdk::kFused) {   // 8 states per lane where a whole block fits TMEM
+            if (a.K == 4) return launch<IO, N, bdk::kFused, 4, 8>(a, batch, st, 1, pdl);
+            if (a.K == 16) return launch<IO, N, bdk::kFused, 16, 8>(a, batch, st, 1, pdl);
+        }
+    }
+    if (mode == bdk::kForwardOnly) return launch<IO, N, bdk::kForwardOnly, 0>(a, batch, st, gz, pdl);
+    if (mode == bdk::kLong) return launch<IO, N, bdk::kLong, 0>(a, batch, st, 1, pdl);
+    if (mode == bdk::kLongFused) return launch<IO, N, bdk::kLongFused, 0>(a, batch, st, 1, pdl);
+    if (mode == bdk::kReverseAcc) return launch<IO, N, bdk::kReverseAcc, 0>(a, batch, st, 1, pdl);
     switch (a.K) {
-        case 4: return launch<IO, N, bdk::kFused, 4>(a, batch, st);
-        case 16: return launch<IO, N, bdk::kFused, 16>(a, batch, st);
-        case 32: return launch<IO, N, bdk::kFused, 32>(a, batch, st);
-        default: return launch<IO, N, bdk::kFused, 0>(a, batch, st);
+        case 4: return launch<IO, N, bdk::kFused, 4>(a, batch, st, 1, pdl);
+        case 16: return launch<IO, N, bdk::kFused, 16>(a, batch, st, 1, pdl);
+        case 32: return launch<IO, N, bdk::kFused, 32>(a, batch, st, 1, pdl);
+        default: return launch<IO, N, bdk::kFused, 0>(a, batch, st, 1, pdl);
     }
 }
 
@@ -187,23 +211,59 @@ int run(Op op, const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, 
     bool thin = false;
     if ((op == kStep || (op == kCommit && y)) && mode == bdk::kFused && dm->d_state == 16)
         thin = dm->batch * ((dm->d_inner + bdk::kCh - 1) / bdk::kCh) <= device_sm_count();
+    // block steps and commits are short, back-to-back launches: overlap each
+    // one's launch with the end of the kernel before it
+    const bool pdl = op == kStep || op == kCommit;
     if (dm->io_dtype == BDSCAN_BF16)
-        return dm->d_state == 16 ? dispatch_mode<__nv_bfloat16, 16>(mode, a, dm->batch, st, gz, thin)
-                                 : dispatch_mode<__nv_bfloat16, 64>(mode, a, dm->batch, st, gz);
-    return dm->d_state == 16 ? dispatch_mode<float, 16>(mode, a, dm->batch, st, gz, thin)
-                             : dispatch_mode<float, 64>(mode, a, dm->batch, st, gz);
+        return dm->d_state == 16 ? dispatch_mode<__nv_bfloat16, 16>(mode, a, dm->batch, st, gz, thin, pdl)
+                                 : dispatch_mode<__nv_bfloat16, 64>(mode, a, dm->batch, st, gz, false, pdl);
+    return dm->d_state == 16 ? dispatch_mode<float, 16>(mode, a, dm->batch, st, gz, thin, pdl)
+                             : dispatch_mode<float, 64>(mode, a, dm->batch, st, gz, false, pdl);
+}
+
+// Resident CTAs per SM of the forward-only scan kernel (both passes of the
+// time-chunked prefill run it), queried once per device; without a device the
+// value the kernels reach on sm_100 (3 at N = 16, 1 at N = 64).
+template <class IO, int N>
+int forward_only_ctas_per_sm() {
+    static std::atomic<int> cache[64] = {};
+    const int fallback = N == 16 ? 3 : 1;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fallback;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
+        using CF = bdk::Cfg<N, bdk::kForwardOnly, 0>;
+        using LY = bdk::Layout<IO, N, bdk::kForwardOnly, 0>;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bdk::bdscan_kernel<IO, N, bdk::kForwardOnly, 0>,
+                                                          CF::THREADS, LY::base_bytes) != cudaSuccess || n <= 0) {
+            (void)cudaGetLastError();
+            n = fallback;
+        }
+        cache[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
+int forward_only_slots(const bdscan_dims *dm) {
+    const int per_sm = dm->io_dtype == BDSCAN_BF16
+                           ? (dm->d_state == 16 ? forward_only_ctas_per_sm<__nv_bfloat16, 16>()
+                                                : forward_only_ctas_per_sm<__nv_bfloat16, 64>())
+                           : (dm->d_state == 16 ? forward_only_ctas_per_sm<float, 16>()
+                                                : forward_only_ctas_per_sm<float, 64>());
+    return per_sm * device_sm_count();
 }
 
 // Chunk plan of the time-chunked prefill. Chunks cost a second pass, so they
 // are used only when the (batch, 32-channel) rows alone give fewer CTAs than
-// the device has SMs; then enough chunks that the CTAs fill the device about
-// three deep, at most 64 chunks and at least 256 tokens per chunk. The chunk
-// length is a multiple of 16 tokens.
+// the device has SMs; then as many chunks as keep all CTAs resident in one
+// wave (rows x chunks <= SMs x resident CTAs per SM: a second, partial wave
+// would nearly double the time), at most 64 chunks and at least 256 tokens per
+// chunk. The chunk length is a multiple of 16 tokens.
 Chunking chunk_plan(const bdscan_dims *dm) {
     Chunking c;
     const int sms = device_sm_count();
     const int64_t row_ctas = dm->batch * ((dm->d_inner + bdk::kCh - 1) / bdk::kCh);
-    int64_t g = (row_ctas > 0 && row_ctas < sms) ? (3 * (int64_t)sms + row_ctas - 1) / row_ctas : 1;
+    int64_t g = (row_ctas > 0 && row_ctas < sms) ? forward_only_slots(dm) / row_ctas : 1;
     const int64_t gmax_len = dm->seqlen / 256 > 0 ? dm->seqlen / 256 : 1;
     if (g > 64) g = 64;
     if (g > gmax_len) g = gmax_len;

@@ -83,7 +83,7 @@ struct BwdLayout {
     static constexpr int xb = TT * kCh * (int)sizeof(IO);   // one x / dt / z / dy tile
     static constexpr int bb = TT * N * (int)sizeof(IO);     // one B / C tile
     static constexpr int stage = 4 * xb + 2 * bb;
-    static constexpr int dq = CF::S * stage;                // float4 (delta, delta*x, ds, 0)  [TT][32]
+    static constexpr int dq = CF::S * stage;                // float4 (delta, delta*x, ds, d delta/d dt) [TT][32]
     static constexpr int bf = dq + TT * kCh * 16;           // float B  [TT][N]
     static constexpr int cf = bf + TT * N * 4;              // float C  [TT][N]
     static constexpr int red = cf + TT * N * 4;             // float [3][W][TT][32]: P, Q, S partials
@@ -277,10 +277,11 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
             for (int e = tid; e < TT * kCh; e += NT) {
                 const float xv = to_f32(xs[e]);
                 const float dr = to_f32(dts[e]);
-                const float dl = a.dt_softplus ? softplus_f32(dr) : dr;
+                float sg = 1.f;   // d delta / d dt
+                const float dl = a.dt_softplus ? softplus_sigmoid_f32(dr, sg) : dr;
                 const float dyv = to_f32(dys[e]);
                 const float dsv = gated ? __fmul_rn(dyv, silu_f32(to_f32(zs[e]))) : dyv;
-                dq[e] = make_float4(dl, __fmul_rn(dl, xv), dsv, 0.f);
+                dq[e] = make_float4(dl, __fmul_rn(dl, xv), dsv, sg);
             }
             constexpr int EPC = 16 / (int)sizeof(IO);
             for (int e = tid; e < TT * N / EPC; e += NT) {
@@ -302,15 +303,27 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
             nu2[1] = make_float2(nv.z, nv.w);
         }
 
+        // A tile of a long-block segment is full whenever the block length is a
+        // multiple of the tile, and holds at most the block's first token (at 0)
+        // and its last (at tlen - 1): those tiles run both sweeps without
+        // per-token guards, the block-start and block-end resets hoisted.
+        const bool fast = longb && tlen == TT;
+
         // ---- forward sweep over the tile (phase 1: state only; phase 2: into TMEM)
+        auto fwd_sweep = [&](auto fast_tag, auto store_tag) {
+            constexpr bool FAST = decltype(fast_tag)::value, STORE = decltype(store_tag)::value;
+            if (FAST && (smask & 1u)) {
+                nu2[0] = f2(0.f);
+                nu2[1] = f2(0.f);
+            }
 #pragma unroll
         for (int t = 0; t < TT; ++t) {
-            if (t < tlen) {
+            if (FAST || t < tlen) {
                 const float4 q4 = dqc[t * kCh];
                 const float4 Cv = *reinterpret_cast<const float4 *>(Cw + t * N);
                 float at[NPT], bq[NPT];
                 decay_input<NPT>(al, make_float2(q4.x, q4.y), Bw + t * N, at, bq);
-                if ((smask >> t) & 1u) {
+                if (!FAST && ((smask >> t) & 1u)) {
                     nu2[0] = f2(0.f);
                     nu2[1] = f2(0.f);
                 }
@@ -329,11 +342,19 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
                     nu2[p] = __fmul2_rn(a2, mu2);
                     h2[p] = __ffma2_rn(a2, h2[p], b2);
                 }
-                if (!tl.ph1) {
+                if (STORE) {
                     tmem_st8(tw + t * 16, va);
                     tmem_st8(tw + t * 16 + 8, vh);
                 }
             }
+        }
+        };
+        if (tl.ph1) {
+            if (fast) fwd_sweep(std::true_type{}, std::false_type{});
+            else fwd_sweep(std::false_type{}, std::false_type{});
+        } else {
+            if (fast) fwd_sweep(std::true_type{}, std::true_type{});
+            else fwd_sweep(std::false_type{}, std::true_type{});
         }
         if (tl.ph1) {
             if (tl.i + 1 < ntb - 1) {
@@ -346,15 +367,24 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
         tmem_wait_st();
 
         // ---- phase 2 backward sweep: the adjoint chains --------------------------
-        {
+        auto bwd_sweep = [&](auto fast_tag, auto gated_tag) {
+            constexpr bool FAST = decltype(fast_tag)::value, GATED = decltype(gated_tag)::value;
+            // h_t of the token being processed: the forward sweep's last state at
+            // the tile end, then each token's h_{t-1} (the same packed FMA made them)
+            float2 hc2[2] = {h2[0], h2[1]};
             float va[8], vh[8];
-            tmem_ld8(tw + (tlen - 1) * 16, va);
-            tmem_ld8(tw + (tlen - 1) * 16 + 8, vh);
+            const int tl1 = FAST ? TT - 1 : tlen - 1;
+            tmem_ld8(tw + tl1 * 16, va);
+            tmem_ld8(tw + tl1 * 16 + 8, vh);
             tmem_wait_ld(va, vh);
+            if (FAST && ((emask >> (TT - 1)) & 1u)) {
+                g2[0] = f2(0.f);
+                g2[1] = f2(0.f);
+            }
             float *redw = red + (warp * TT) * kCh + c;   // [q][warp][t][lane]
 #pragma unroll
             for (int t = TT - 1; t >= 0; --t) {
-                if (t < tlen) {
+                if (FAST || t < tlen) {
                     float na[8], nh[8];
                     if (t > 0) {   // next token's row, read while this one computes
                         tmem_ld8(tw + (t - 1) * 16, na);
@@ -363,7 +393,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
                     const float4 q4 = dqc[t * kCh];   // delta, delta*x, ds
                     const float4 Bv = *reinterpret_cast<const float4 *>(Bw + t * N);
                     const float4 Cv = *reinterpret_cast<const float4 *>(Cw + t * N);
-                    if ((emask >> t) & 1u) {
+                    if (!FAST && ((emask >> t) & 1u)) {
                         g2[0] = f2(0.f);
                         g2[1] = f2(0.f);
                     }
@@ -381,12 +411,12 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
                         const float2 db2 = __fadd2_rn(lam2, mu2);
                         const float2 da2 = __ffma2_rn(mu2, g2[p], __fmul2_rn(lam2, hp2));
                         const float2 gn2 = __ffma2_rn(a2, g2[p], b2);
-                        const float2 hn2 = __ffma2_rn(a2, hp2, b2);
-                        const float2 hg2 = __fadd2_rn(hn2, gn2);
+                        const float2 hg2 = __fadd2_rn(hc2[p], gn2);
+                        hc2[p] = hp2;
                         const float2 qa2 = __fmul2_rn(da2, a2);
                         P2 = __ffma2_rn(db2, B2[p], P2);
                         Q2 = __ffma2_rn(qa2, Av2[p], Q2);
-                        if (gated) S2 = __ffma2_rn(C2[p], hg2, S2);
+                        if (GATED) S2 = __ffma2_rn(C2[p], hg2, S2);
                         dA2[p] = __ffma2_rn(qa2, dl2, dA2[p]);
                         dB2[p] = __fmul2_rn(db2, dlx2);
                         dC2[p] = __fmul2_rn(ds2, hg2);
@@ -395,7 +425,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
                     }
                     redw[t * kCh] = __fadd_rn(P2.x, P2.y);
                     redw[(W * TT + t) * kCh] = __fadd_rn(Q2.x, Q2.y);
-                    if (gated) redw[(2 * W * TT + t) * kCh] = __fadd_rn(S2.x, S2.y);
+                    if (GATED) redw[(2 * W * TT + t) * kCh] = __fadd_rn(S2.x, S2.y);
                     float *brow = bcr + (t * kCh + c) * BR + n0;
                     *reinterpret_cast<float4 *>(brow) = make_float4(dB2[0].x, dB2[0].y, dB2[1].x, dB2[1].y);
                     *reinterpret_cast<float4 *>(brow + N) = make_float4(dC2[0].x, dC2[0].y, dC2[1].x, dC2[1].y);
@@ -406,6 +436,13 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
                     }
                 }
             }
+        };
+        if (fast) {
+            if (gated) bwd_sweep(std::true_type{}, std::true_type{});
+            else bwd_sweep(std::true_type{}, std::false_type{});
+        } else {
+            if (gated) bwd_sweep(std::false_type{}, std::true_type{});
+            else bwd_sweep(std::false_type{}, std::false_type{});
         }
         __syncthreads();
 
@@ -428,7 +465,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
                     const float xv = to_f32(xs[e]);
                     const float dxv = __fmaf_rn(q4.x, P, __fmul_rn(dfac, q4.z));
                     float ddl = __fmaf_rn(xv, P, Q);
-                    if (a.dt_softplus) ddl = __fmul_rn(ddl, sigmoid_f32(to_f32(dts[e])));
+                    if (a.dt_softplus) ddl = __fmul_rn(ddl, q4.w);
                     const int64_t go = (b * L + tl.t0 + t) * a.D + d;
                     IO o;
                     from_f32(dxv, o);

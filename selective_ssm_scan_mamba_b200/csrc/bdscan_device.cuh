@@ -38,8 +38,7 @@ __device__ __forceinline__ void from_f32(float v, __nv_bfloat16 &o) { o = __floa
 // log1p(u) = u * P(u) with P a degree-9 polynomial fitted to log1p(u)/u on
 // [0, 1] (relative-error weighted least squares on Chebyshev nodes); about
 // 1.5 ulp over the whole range, including u -> 0 where log1p(u) ~ u.
-__device__ __forceinline__ float softplus_f32(float v) {
-    const float u = ex2_approx(__fmul_rn(-fabsf(v), kLog2e));
+__device__ __forceinline__ float softplus_from_u(float v, float u) {
     float p = -0.003244000254198909f;
     p = __fmaf_rn(p, u, 0.01985134929418564f);
     p = __fmaf_rn(p, u, -0.05695932358503342f);
@@ -51,6 +50,16 @@ __device__ __forceinline__ float softplus_f32(float v) {
     p = __fmaf_rn(p, u, -0.4999990165233612f);
     p = __fmaf_rn(p, u, 1.0f);
     return __fadd_rn(fmaxf(v, 0.f), __fmul_rn(u, p));
+}
+__device__ __forceinline__ float softplus_f32(float v) {
+    return softplus_from_u(v, ex2_approx(__fmul_rn(-fabsf(v), kLog2e)));
+}
+// softplus(v) (the same bits as softplus_f32) and its derivative
+// sigmoid(v) = (v >= 0 ? 1 : u) / (1 + u), from the one exp u = e^{-|v|}
+__device__ __forceinline__ float softplus_sigmoid_f32(float v, float &sig) {
+    const float u = ex2_approx(__fmul_rn(-fabsf(v), kLog2e));
+    sig = __fmul_rn(v >= 0.f ? 1.f : u, rcp_approx(__fadd_rn(1.f, u)));
+    return softplus_from_u(v, u);
 }
 
 // silu(z) = z / (1 + e^{-z})
@@ -129,6 +138,29 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
                  : "r"(taddr)
                  : "memory");
 }
+// 16 consecutive 32-bit columns of this lane's row
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16};" ::"r"(taddr),
+        "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]),
+        "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]), "=f"(v[8]),
+          "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+// width-generic forms (8 or 16 columns)
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const float (&v)[8]) { tmem_st8(taddr, v); }
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const float (&v)[16]) { tmem_st16(taddr, v); }
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[8]) { tmem_ld8(taddr, v); }
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[16]) { tmem_ld16(taddr, v); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 // Wait for this thread's outstanding TMEM loads. The loaded registers pass
 // through the instruction so that no use of them can be scheduled before it.
@@ -136,6 +168,15 @@ __device__ __forceinline__ void tmem_wait_ld(float (&u)[8], float (&v)[8]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+f"(u[0]), "+f"(u[1]), "+f"(u[2]), "+f"(u[3]), "+f"(u[4]), "+f"(u[5]), "+f"(u[6]), "+f"(u[7]),
                    "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7])
+                 :
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld(float (&u)[16], float (&v)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+f"(u[0]), "+f"(u[1]), "+f"(u[2]), "+f"(u[3]), "+f"(u[4]), "+f"(u[5]), "+f"(u[6]), "+f"(u[7]),
+                   "+f"(u[8]), "+f"(u[9]), "+f"(u[10]), "+f"(u[11]), "+f"(u[12]), "+f"(u[13]), "+f"(u[14]), "+f"(u[15]),
+                   "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
+                   "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15])
                  :
                  : "memory");
 }

@@ -48,6 +48,8 @@
 //            element).
 #pragma once
 
+#include <type_traits>
+
 #include "bdscan_device.cuh"
 
 namespace bdk {
@@ -79,12 +81,14 @@ struct ScanArgs {
     int32_t K, dt_softplus;
 };
 
-// NPTV = states per lane: 4 (one warp per 4 states) everywhere but the thin
-// block-step variant, 1 state per lane (16 warps per CTA at N = 16), which a
-// block step of too few channels to fill the GPU uses: its 32 tokens are a
-// latency chain, and a quarter of the per-token work per warp shortens it.
-// Prefills of too few channels get their parallelism from time chunks
-// (bdscan_prefill_chunked) instead.
+// NPT = states per lane: 4 (one warp per 4 states) by default; 8 for the
+// whole-block fused variants at N = 64 (8 warps per CTA: half the per-element
+// shared-memory reads of delta and of the readout partials, twice the
+// independent work per warp); 1 for the thin block-step variant (16 warps per
+// CTA at N = 16), which a block step of too few channels to fill the GPU uses:
+// its 32 tokens are a latency chain, and a quarter of the per-token work per
+// warp shortens it. Prefills of too few channels get their parallelism from
+// time chunks (bdscan_prefill_chunked) instead.
 template <int N, int MODE, int KC, int NPTV = 4>
 struct Cfg {
     static constexpr int NPT = NPTV;
@@ -96,20 +100,25 @@ struct Cfg {
     static constexpr int SPAN = MODE == kFused ? (KC > 0 ? KC : T) : 16;
     static constexpr bool KEEP_B = SPAN <= 16 && N == 16;                        // keep b for phase C
     static constexpr int PER = T / W > 0 ? T / W : 1;                            // readout tokens per warp
+    static constexpr int PV = PER >= 4 ? 4 : PER;                                // readout vector width
     // whole-block fused variants (and the long fused mode, span by span) keep a
-    // span's decays and inputs in TMEM (8 columns per token: a[4], b[4]). Warp
-    // w uses lane quadrant w % 4 and column range (w / 4) * WCOLS; a CTA's
-    // columns fit the SM's 512 at the residency each variant reaches (N = 16:
-    // 3 CTAs x 128 for spans of 16, 2 CTAs x 256 for K = 32; N = 64: 1 x 512).
+    // span's decays and inputs in TMEM (2 * NPT columns per token: a[NPT],
+    // b[NPT]). Warp w uses lane quadrant w % 4 and column range (w / 4) * WCOLS;
+    // a CTA's columns fit the SM's 512 at the residency each variant reaches
+    // (N = 16: 3 CTAs x 128 for spans of 16, 2 CTAs x 256 for K = 32; N = 64,
+    // K = 16: 1 x 512; N = 64, K = 4: 2 x 128).
     static constexpr int WCOLS = SPAN * 2 * NPT;
     static constexpr int TNEED = (W / 4) * WCOLS;
-    static constexpr bool TMEM = ((MODE == kFused && KC > 0) || MODE == kLongFused) && W % 4 == 0 && NPT == 4 &&
-                                 TNEED <= 512;
+    static constexpr bool TMEM = ((MODE == kFused && KC > 0) || MODE == kLongFused) && W % 4 == 0 &&
+                                 (NPT == 4 || (NPT == 8 && MODE == kFused)) && TNEED <= 512;
     static constexpr int TCOLS = TNEED <= 32 ? 32 : (TNEED <= 64 ? 64 : (TNEED <= 128 ? 128 : (TNEED <= 256 ? 256 : 512)));
     // registers: the four N = 16 state-group warps of a CTA sit on the SM's four
     // sub-partitions, so 3 resident CTAs = 3 warps per sub-partition (<= 168
     // registers), enough for a 12288-channel batch in one wave on 148 SMs.
-    static constexpr int MINB = THREADS >= 512 ? 1 : ((T == 16 || KC == 16 || MODE == kLongFused) ? 3 : 2);
+    // (8 states per lane: 2 CTAs, up to 128 registers, where TMEM allows)
+    static constexpr int MINB0 = THREADS >= 512 ? 1 : NPT == 8 ? 2
+                               : ((T == 16 || KC == 16 || MODE == kLongFused) ? 3 : 2);
+    static constexpr int MINB = (TMEM && 512 / TCOLS < MINB0) ? 512 / TCOLS : MINB0;
     static_assert(N % NPT == 0 && W <= 32, "state split");
 };
 
@@ -118,18 +127,17 @@ template <class IO, int N, int MODE, int KC, int NPTV = 4>
 struct Layout {
     using CF = Cfg<N, MODE, KC, NPTV>;
     static constexpr int T = CF::T, S = CF::S, W = CF::W;
-    static constexpr int RP = T + 4;                       // padded row of the readout buffer
     static constexpr int xb = T * kCh * (int)sizeof(IO);   // one x / dt / z tile
     static constexpr int bb = T * N * (int)sizeof(IO);     // one B / C tile
     static constexpr int stage = 3 * xb + 2 * bb;
     static constexpr int dd = S * stage;                   // float2 (delta, delta*x)   [T][32]
     static constexpr int bf = dd + T * kCh * 8;            // float B                  [T][N]
     static constexpr int cf = bf + T * N * 4;              // float C                  [T][N]
-    static constexpr int red = cf + T * N * 4;             // float partial readouts   [W][32][RP]
-    static constexpr int yrev = red + W * kCh * RP * 4;    // float reverse readout [K][32] (long), or the
+    static constexpr int red = cf + T * N * 4;             // float partial readouts   [W][T/PV][32][PV]
+    static constexpr int yrev = red + W * T * kCh * 4;     // float reverse readout [K][32] (long), or the
                                                            // float4 span checkpoints [spans-1][W][32] (long fused)
     static constexpr int base_bytes = yrev;
-    static_assert(xb % 16 == 0 && bb % 16 == 0 && (RP * 4) % 16 == 0, "16-byte rows");
+    static_assert(xb % 16 == 0 && bb % 16 == 0, "16-byte rows");
 };
 
 // ---- per-lane arithmetic on NPT states (NPT = 1, 2 or 4) -----------------------
@@ -182,7 +190,10 @@ __device__ __forceinline__ float scan_step(float (&st)[NPT], const float (&a)[NP
         st[0] = __fmaf_rn(a[0], st[0], bq[0]);
         return __fmul_rn(Cn[0], st[0]);
     } else {
-        float2 acc = make_float2(0.f, 0.f);
+        // readout partial: at 8 states per lane two packed accumulators (even /
+        // odd state pairs) keep the dependent chain short
+        constexpr int NA = NPT >= 8 ? 2 : 1;
+        float2 acc[NA];
 #pragma unroll
         for (int p = 0; p < NPT / 2; ++p) {
             const float2 s2 = __ffma2_rn(make_float2(a[2 * p], a[2 * p + 1]), make_float2(st[2 * p], st[2 * p + 1]),
@@ -190,9 +201,11 @@ __device__ __forceinline__ float scan_step(float (&st)[NPT], const float (&a)[NP
             st[2 * p] = s2.x;
             st[2 * p + 1] = s2.y;
             const float2 c2 = make_float2(Cn[2 * p], Cn[2 * p + 1]);
-            acc = p == 0 ? __fmul2_rn(c2, s2) : __ffma2_rn(c2, s2, acc);
+            const int q = p % NA;
+            acc[q] = p < NA ? __fmul2_rn(c2, s2) : __ffma2_rn(c2, s2, acc[q]);
         }
-        return __fadd_rn(acc.x, acc.y);
+        if constexpr (NA == 2) acc[0] = __fadd2_rn(acc[0], acc[1]);
+        return __fadd_rn(acc[0].x, acc[0].y);
     }
 }
 
@@ -240,7 +253,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
     using CF = Cfg<N, MODE, KC, NPTV>;
     using LY = Layout<IO, N, MODE, KC, NPTV>;
     constexpr int NPT = CF::NPT, W = CF::W, NT = CF::THREADS, T = CF::T, S = CF::S, SPAN = CF::SPAN;
-    constexpr int RP = LY::RP, PER = CF::PER;
+    constexpr int PER = CF::PER, PV = CF::PV;
     constexpr bool KEEP_B = CF::KEEP_B;
     static_assert(T % SPAN == 0, "spans tile the tile");
     static_assert(SPAN % 2 == 0 || !(MODE == kFused && KC > 0), "interleaved chains pair tokens");
@@ -266,6 +279,13 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
     const int64_t tend = chunked ? (tbeg + a.chunk_len < L ? tbeg + a.chunk_len : L) : L;
     const bool gated = a.z != nullptr;
     const bool want_y = a.y != nullptr;
+    // Programmatic dependent launch (block steps and commits are launched with
+    // it): let the next kernel of the stream start launching now, and wait
+    // until the previous one has completed, its memory visible, before the
+    // first global access (read or write). Both are no-ops for a kernel
+    // launched without the attribute.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const float dskip = dvalid ? a.Dskip[d] : 0.f;
     const float dfac = MODE == kForwardOnly ? dskip : __fmul_rn(2.f, dskip);
 
@@ -359,7 +379,8 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
         if (s < nsteps) {
             int64_t t0; int tlen; bool rv, fr;
             tile_of(s, t0, tlen, rv, fr);
-            const bool state_only = MODE == kLongFused && rv;   // the g-only reverse sweep reads no C, z
+            // the g-only reverse sweep and the chunk-summary pass read no C, z
+            const bool state_only = (MODE == kLongFused && rv) || (MODE == kForwardOnly && a.chunk_pass == 1);
             stage_tile<IO, N, T, NT>(smem + (s % S) * LY::stage, a, b, d0, t0, tlen, gated && !state_only,
                                      !state_only);
         }
@@ -372,7 +393,10 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
     auto write_boundary = [&](int64_t tok_end) {   // state after token tok_end (a block end)
         if (bnd_ptr) {
             float *p = bnd_ptr + ((tok_end + 1) / K - 1) * bnd_stride;
-            if constexpr (NPT == 4) *reinterpret_cast<float4 *>(p) = make_float4(h[0], h[1], h[2], h[3]);
+            if constexpr (NPT == 8) {
+                *reinterpret_cast<float4 *>(p) = make_float4(h[0], h[1], h[2], h[3]);
+                *reinterpret_cast<float4 *>(p + 4) = make_float4(h[4], h[5], h[6], h[7]);
+            } else if constexpr (NPT == 4) *reinterpret_cast<float4 *>(p) = make_float4(h[0], h[1], h[2], h[3]);
             else if constexpr (NPT == 2) *reinterpret_cast<float2 *>(p) = make_float2(h[0], h[1]);
             else p[0] = h[0];
         }
@@ -428,7 +452,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
         // ---- the scan over this tile --------------------------------------------
         float yp[T];
         uint32_t endmask = 0;   // block ends inside the tile (runtime-K and forward-only)
-        if (MODE == kForwardOnly || (MODE == kFused && KC == 0)) {
+        if ((MODE == kForwardOnly && a.boundary) || (MODE == kFused && KC == 0)) {
             for (int64_t e = K - 1 - (t0 % K); e < tlen; e += K) endmask |= 1u << e;   // block ends in the tile
         } else if (MODE == kLong) {
             if (!rev && (t0 + tlen) % K == 0) endmask = 1u << (tlen - 1);
@@ -513,32 +537,35 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
                     }
                 }
                 if constexpr (CF::TMEM) {
+                    constexpr int TV = 2 * NPT;   // TMEM columns per token: a[NPT], b[NPT]
                     // (A) a and b of every token of the block into this warp's TMEM lanes
 #pragma unroll
                     for (int i = 0; i < SPAN; ++i) {
-                        float at4[NPT], bq4[NPT], v[8];
+                        float at4[NPT], bq4[NPT], v[TV];
                         decay_input<NPT>(al, ddc[(s0 + i) * kCh], Bw + (s0 + i) * N, at4, bq4);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) { v[j] = at4[j]; v[4 + j] = bq4[j]; }
-                        tmem_st8(tmem_w + i * 8, v);
+                        for (int j = 0; j < NPT; ++j) { v[j] = at4[j]; v[NPT + j] = bq4[j]; }
+                        tmem_st(tmem_w + i * TV, v);
                     }
                     tmem_wait_st();
                     // (B)+(C), reading step i+1's operands while step i computes
-                    float cf[8], cr[8];
-                    tmem_ld8(tmem_w + 0, cf);
-                    tmem_ld8(tmem_w + (SPAN - 1) * 8, cr);
+                    float cf[TV], cr[TV];
+                    tmem_ld(tmem_w + 0, cf);
+                    tmem_ld(tmem_w + (SPAN - 1) * TV, cr);
                     tmem_wait_ld(cf, cr);
 #pragma unroll
                     for (int i = 0; i < SPAN; ++i) {
                         const int tf = s0 + i, ir = SPAN - 1 - i, tr = s0 + ir;
-                        float nf[8], nr[8];
+                        float nf[TV], nr[TV];
                         if (i + 1 < SPAN) {
-                            tmem_ld8(tmem_w + (i + 1) * 8, nf);
-                            tmem_ld8(tmem_w + (ir - 1) * 8, nr);
+                            tmem_ld(tmem_w + (i + 1) * TV, nf);
+                            tmem_ld(tmem_w + (ir - 1) * TV, nr);
                         }
                         float af[NPT], bfq[NPT], ar[NPT], brq[NPT];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) { af[j] = cf[j]; bfq[j] = cf[4 + j]; ar[j] = cr[j]; brq[j] = cr[4 + j]; }
+                        for (int j = 0; j < NPT; ++j) {
+                            af[j] = cf[j]; bfq[j] = cf[NPT + j]; ar[j] = cr[j]; brq[j] = cr[NPT + j];
+                        }
                         const float vf = scan_step<NPT>(h, af, bfq, Cw + tf * N);
                         const float vr = scan_step<NPT>(gs, ar, brq, Cw + tr * N);
                         if (i < SPAN / 2) {
@@ -551,7 +578,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
                         if (i + 1 < SPAN) {
                             tmem_wait_ld(nf, nr);
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) { cf[j] = nf[j]; cr[j] = nr[j]; }
+                            for (int j = 0; j < TV; ++j) { cf[j] = nf[j]; cr[j] = nr[j]; }
                         }
                     }
                 } else {
@@ -605,16 +632,71 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
                 if (t < tlen) {
                     float at_[NPT], bq_[NPT];
                     decay_input<NPT>(al, ddc[t * kCh], Bw + t * N, at_, bq_);
+                    if constexpr (NPT % 2 == 0) {
 #pragma unroll
-                    for (int j = 0; j < NPT; ++j) {
-                        h[j] = __fmaf_rn(at_[j], h[j], bq_[j]);
-                        pdec[j] = __fmul_rn(pdec[j], at_[j]);
+                        for (int p = 0; p < NPT / 2; ++p) {
+                            const float2 a2 = make_float2(at_[2 * p], at_[2 * p + 1]);
+                            const float2 h2 = __ffma2_rn(a2, make_float2(h[2 * p], h[2 * p + 1]),
+                                                         make_float2(bq_[2 * p], bq_[2 * p + 1]));
+                            const float2 p2 = __fmul2_rn(make_float2(pdec[2 * p], pdec[2 * p + 1]), a2);
+                            h[2 * p] = h2.x; h[2 * p + 1] = h2.y;
+                            pdec[2 * p] = p2.x; pdec[2 * p + 1] = p2.y;
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < NPT; ++j) {
+                            h[j] = __fmaf_rn(at_[j], h[j], bq_[j]);
+                            pdec[j] = __fmul_rn(pdec[j], at_[j]);
+                        }
                     }
                 }
-                yp[t] = 0.f;
+            }
+        } else if (MODE == kForwardOnly) {
+            // forward-only scan (prefill, commit without y, time-chunked pass 2):
+            // (A) decays and inputs of a span, (B) the chain with its readout
+            // partials. Full spans (all but a ragged last tile) run without
+            // per-token guards; block-end states are tested for only when the
+            // caller asked for them.
+            const bool wb = endmask != 0 && bnd_ptr != nullptr;
+            auto fwd_span = [&](int s0, auto whole_tag) {
+                constexpr bool WHOLE = decltype(whole_tag)::value;
+                constexpr int NB = KEEP_B ? SPAN : 1;
+                float at[SPAN][NPT];
+                float bt[NB][NPT];
+#pragma unroll
+                for (int i = 0; i < SPAN; ++i) {   // (A); rows past a ragged end are computed, never used
+                    float bq[NPT];
+                    decay_input<NPT>(al, ddc[(s0 + i) * kCh], Bw + (s0 + i) * N, at[i], bq);
+                    if (KEEP_B) {
+#pragma unroll
+                        for (int j = 0; j < NPT; ++j) bt[KEEP_B ? i : 0][j] = bq[j];
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < SPAN; ++i) {   // (B)
+                    const int t = s0 + i;
+                    if (WHOLE || t < tlen) {
+                        float bq[NPT];
+                        if (KEEP_B) {
+#pragma unroll
+                            for (int j = 0; j < NPT; ++j) bq[j] = bt[KEEP_B ? i : 0][j];
+                        } else {
+                            input_only<NPT>(ddc[t * kCh].y, Bw + t * N, bq);
+                        }
+                        yp[t] = scan_step<NPT>(h, at[i], bq, Cw + t * N);
+                        if (wb && ((endmask >> t) & 1u)) write_boundary(t0 + t);
+                    } else {
+                        yp[t] = 0.f;
+                    }
+                }
+            };
+#pragma unroll
+            for (int sp = 0; sp < T / SPAN; ++sp) {
+                if (sp * SPAN + SPAN <= tlen) fwd_span(sp * SPAN, std::true_type{});
+                else fwd_span(sp * SPAN, std::false_type{});
             }
         } else {
-            // forward-only, and fused with a runtime block length (<= 32)
+            // fused with a runtime block length (<= 32)
             constexpr bool REV = MODE == kFused;
             constexpr int NB = KEEP_B ? SPAN : 1;
 #pragma unroll
@@ -681,12 +763,21 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
         // ---- readout: the W state-group partials of every (token, channel) -------
         // (a forward-only pass without y -- commit, chunked pass 1 -- has none)
         if (MODE == kForwardOnly && !want_y) continue;
+        // partials layout [W][T/PV][32][PV]: a lane's PV consecutive tokens are
+        // one vector, and a warp's 32 lanes touch 32 consecutive vectors on both
+        // the write and the read side (no bank conflicts)
         {
-            float *rrow = red + (warp * kCh + c) * RP;   // this warp's partials for channel c
+            float *wrow = red + (warp * (T / PV) * kCh + c) * PV;
 #pragma unroll
-            for (int q = 0; q < T / 4; ++q)
-                *reinterpret_cast<float4 *>(rrow + 4 * q) =
-                    make_float4(yp[4 * q], yp[4 * q + 1], yp[4 * q + 2], yp[4 * q + 3]);
+            for (int q = 0; q < T / PV; ++q) {
+                float *dst = wrow + q * kCh * PV;
+                if constexpr (PV == 4)
+                    *reinterpret_cast<float4 *>(dst) = make_float4(yp[4 * q], yp[4 * q + 1], yp[4 * q + 2], yp[4 * q + 3]);
+                else if constexpr (PV == 2)
+                    *reinterpret_cast<float2 *>(dst) = make_float2(yp[2 * q], yp[2 * q + 1]);
+                else
+                    dst[0] = yp[q];
+            }
         }
         __syncthreads();
         // warp w finishes tokens [w*PER, (w+1)*PER) of the tile
@@ -696,21 +787,26 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
             for (int i = 0; i < PER; ++i) ysum[i] = 0.f;
 #pragma unroll
             for (int gg = 0; gg < W; ++gg) {
-                const float *rrow = red + (gg * kCh + c) * RP + warp * PER;
-                if constexpr (PER % 4 == 0) {
+                const float *rrow = red + ((gg * (T / PV) + warp * (PER / PV)) * kCh + c) * PV;
 #pragma unroll
-                    for (int q = 0; q < PER / 4; ++q) {
-                        const float4 v = *reinterpret_cast<const float4 *>(rrow + 4 * q);
+                for (int q = 0; q < PER / PV; ++q) {
+                    const float *src = rrow + q * kCh * PV;
+                    if constexpr (PV == 4) {
+                        const float4 v = *reinterpret_cast<const float4 *>(src);
                         const float2 s0 = __fadd2_rn(make_float2(ysum[4 * q], ysum[4 * q + 1]), make_float2(v.x, v.y));
                         const float2 s1 = __fadd2_rn(make_float2(ysum[4 * q + 2], ysum[4 * q + 3]), make_float2(v.z, v.w));
                         ysum[4 * q] = s0.x;
                         ysum[4 * q + 1] = s0.y;
                         ysum[4 * q + 2] = s1.x;
                         ysum[4 * q + 3] = s1.y;
+                    } else if constexpr (PV == 2) {
+                        const float2 v = *reinterpret_cast<const float2 *>(src);
+                        const float2 s0 = __fadd2_rn(make_float2(ysum[2 * q], ysum[2 * q + 1]), v);
+                        ysum[2 * q] = s0.x;
+                        ysum[2 * q + 1] = s0.y;
+                    } else {
+                        ysum[q] = __fadd_rn(ysum[q], src[0]);
                     }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < PER; ++i) ysum[i] = __fadd_rn(ysum[i], rrow[i]);
                 }
             }
             IO *gy = want_y ? static_cast<IO *>(a.y) + (b * L + t0) * a.D + d : nullptr;

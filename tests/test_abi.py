@@ -212,7 +212,7 @@ def test_train_two_stream_checks_both_passes_first(lib):
     assert f(C.byref(d), C.byref(_ins()), C.byref(_ins()), None, None, None, P + 0x800, None, None) == 1
     # y_noisy misaligned
     assert f(C.byref(d), C.byref(_ins()), C.byref(_ins()), None, None, P + 0x604, P + 0x800, None, None) == 3
-    # a block whose checkpoints fit neither long mode (bf16, N = 16: K > 1392 and K > 768)
+    # a block whose checkpoints fit neither long mode (bf16, N = 16: K > 1408 and K > 768)
     d = Dims(1, 2048, 64, 16, 2048, 1, 1)
     assert f(C.byref(d), C.byref(_ins()), C.byref(_ins()), None, None, P + 0x600, P + 0x800, None, None) == 2
 
@@ -237,3 +237,14 @@ def test_prefill_chunked_checks_both_passes_first(lib, noalloc):
     assert call(None, P + 0x604, P + 0x700, None) == 3            # y misaligned
     assert call(P + 0x808, P + 0x600, P + 0x700, None) == 3       # h0 misaligned
     assert call(None, P + 0x600, P + 0x700, P + 0x90c) == 3       # boundary misaligned
+
+
+@cpu_only
+@pytest.mark.parametrize("io,kmax", [(1, 1408), (0, 1216)])
+def test_long_block_limit_at_n16(lib, io, kmax):
+    """The header's longest block at N = 16 (span checkpoints in shared memory;
+    the two-sweep path stops at 768): kmax is accepted (on this CPU-only check
+    the launch itself then fails with BDSCAN_ERR_CUDA), kmax + 16 is
+    BDSCAN_ERR_UNSUPPORTED."""
+    assert _train(lib, Dims(1, kmax, 64, 16, kmax, io, 1), _ins()) == 5
+    assert _train(lib, Dims(1, kmax + 16, 64, 16, kmax + 16, io, 1), _ins()) == 2

@@ -47,9 +47,13 @@ TRAIN_CASES = [
     (1, 128, 16, 64, 64, "bf16", False, True, True),
     (1, 96, 32, 64, 32, "f32", True, True, True),
     (1, 70, 24, 64, 7, "f32", False, True, True),
+    # N = 64 with 8 states per lane (K = 4, 16): several channel tiles, the last ragged
+    (3, 160, 200, 64, 16, "bf16", True, True, True),
+    (2, 100, 104, 64, 4, "f32", True, True, True),
+    (1, 64, 48, 64, 16, "f32", False, False, False),
     # long blocks whose span checkpoints do not fit in shared memory: the two-sweep path
     (1, 512, 16, 64, 512, "bf16", True, True, True),
-    (1, 256, 16, 64, 256, "f32", False, True, True),
+    (1, 288, 16, 64, 288, "f32", False, True, True),
     (1, 200, 24, 16, 100, "bf16", True, True, True),
 ]
 
@@ -97,6 +101,7 @@ STEP_CASES = [
     (1, 32, 64, 16, "bf16", False), (3, 16, 72, 16, "f32", True), (2, 5, 40, 16, "f32", False),
     (1, 48, 64, 16, "bf16", True), (2, 32, 16, 64, "bf16", False), (1, 20, 24, 64, "f32", True),
     (1, 64, 32, 64, "bf16", True), (2, 100, 24, 16, "f32", False),
+    (2, 16, 200, 64, "bf16", True), (3, 4, 72, 64, "f32", False),
 ]
 
 

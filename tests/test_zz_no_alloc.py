@@ -86,13 +86,19 @@ def test_noalloc_matches_workspace_entry_point_on_calls_in_a_row():
             assert torch.equal(out[k], ref[k]), f"seed {s_seed(s)}: {k} differs from the workspace entry point"
 
 
-def test_noalloc_rejects_sizes_beyond_its_scratch():
-    # fake, never dereferenced: the size check returns before any launch
+def test_noalloc_scratch_covers_every_chunk_plan():
+    """The chunk plan keeps every CTA of both passes resident in one wave, so
+    the scratch a plan needs is about 256 bytes x N per resident CTA slot:
+    under 2.5 MB on a 148-SM B200 whatever the sizes, well inside the fixed
+    8 MiB (the entry point's WORKSPACE rejection then never triggers there).
+    Checked on the planner alone, with no device call."""
     bd = _abi()
     lib = bd.raw_library()
-    dims = bd.Dims(1, 8192, 4608, 64, 16, bd.BF16, 1)
-    assert int(lib.bdscan_prefill_chunked_workspace(ct.byref(dims))) > SCRATCH_BYTES
-    P = 0x100000
-    ins = bd.Inputs(P, P + 0x100, P + 0x200, P + 0x300, None, P + 0x400, P + 0x500)
-    rc = lib.bdscan_prefill_chunked_noalloc(ct.byref(dims), ct.byref(ins), None, P + 0x600, P + 0x700, None, None)
-    assert lib.bdscan_status_string(rc).decode().endswith("WORKSPACE"), rc
+    worst = 0
+    for N in (16, 64):
+        for io in (bd.BF16, bd.F32):
+            for batch in (1, 2, 3, 4):
+                for D in range(32, 4768, 32):
+                    dims = bd.Dims(batch, 1 << 20, D, N, 16, io, 1)
+                    worst = max(worst, int(lib.bdscan_prefill_chunked_workspace(ct.byref(dims))))
+    assert 0 < worst <= SCRATCH_BYTES, worst
