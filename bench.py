@@ -50,12 +50,12 @@ PROFILE_TRAFFIC = {"stack350m": os.path.join(ROOT, "profiles", "stack350m_traffi
 
 
 def kernel_source_hash() -> str:
-    """Hash of the code the forward scan kernel is compiled from (its device
-    sources, with comments and whitespace removed: host-side launch code,
-    other kernels and comment edits do not change it)."""
+    """Hash of the code the forward scan kernels are compiled from (their
+    device sources, with comments and whitespace removed: host-side launch
+    code, the backward kernel and comment edits do not change it)."""
     import re
     h = hashlib.sha256()
-    for name in ("bdscan_device.cuh", "bdscan_kernels.cuh"):
+    for name in ("bdscan_device.cuh", "bdscan_kernels.cuh", "bdscan_lag.cuh"):
         src = open(os.path.join(ROOT, "selective_ssm_scan_mamba_b200", "csrc", name)).read()
         src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
         src = re.sub(r"//[^\n]*", " ", src)
@@ -882,7 +882,7 @@ def run_context_parallel(args):
     return 0
 
 
-def _oracle_sample(name):
+def _oracle_sample(name, scale=1):
     """Bounded oracle sample of a workload's timed unit: (inputs, params, what the
     unit is, element-steps of the full unit / of the sample, call). Channels are
     independent, so the cost of the unit is exactly linear in the channels and
@@ -890,14 +890,14 @@ def _oracle_sample(name):
     import oracle
     w = I.WORKLOADS[name]
     if name == "pr1":
-        chans, n_seq, L, op, unit = list(range(w.D)), w.batch, w.L, "train", "train_blocks, 256 tokens"
+        nch, n_seq, L, op, unit = w.D, w.batch, w.L, "train", "train_blocks, 256 tokens"
     elif name == "train":
-        chans, n_seq, L, op, unit = list(range(192)), w.batch, w.L, "train", "train_blocks, 8 x 4096 tokens"
+        nch, n_seq, L, op, unit = 192, w.batch, w.L, "train", "train_blocks, 8 x 4096 tokens"
     elif name == "stack350m":
-        chans, n_seq, L, op, unit = list(range(32)), w.batch, w.L, "train", "24 layers, 16 x 8192 tokens, K = 16"
+        nch, n_seq, L, op, unit = 32, w.batch, w.L, "train", "24 layers, 16 x 8192 tokens, K = 16"
     else:   # inference: the context prefill (forward-only scan) of all sequences
-        chans, n_seq, L, op, unit = list(range(64)), w.batch, 8192, "prefill", \
-            f"prefill of {w.batch} x {w.L} context tokens"
+        nch, n_seq, L, op, unit = 64, w.batch, 8192, "prefill", f"prefill of {w.batch} x {w.L} context tokens"
+    chans = list(range(min(w.D, nch * scale)))   # (scale: one sample's worth per worker)
     s = I.make_sequence(w.seed, n_seq, L, w.D, w.N, w.io, stream="seq" if op == "train" else ("context",),
                         channels=chans)
     p = I.make_params(w.seed, w.D, w.N)
@@ -926,6 +926,8 @@ def baseline_table(bench_path=None) -> str:
         t0 = time.perf_counter()
         fn()
         t1 = (time.perf_counter() - t0) * full / part
+        # all cores: one single-thread sample's worth of channels per worker
+        s, A, Dk, unit, full, part, fn, op = _oracle_sample(name, scale=os.cpu_count() or 1)
         pool = OraclePool(s, A, Dk, w.K, op=op)
         try:
             ta = pool.step() * full / part

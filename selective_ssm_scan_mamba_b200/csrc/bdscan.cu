@@ -7,6 +7,7 @@
 #include "../../include/bdscan.h"
 #include "bdscan_backward.cuh"
 #include "bdscan_kernels.cuh"
+#include "bdscan_lag.cuh"
 
 namespace {
 
@@ -98,6 +99,28 @@ int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz =
     return BDSCAN_OK;
 }
 
+// The lagged whole-block pass (bdscan_lag_kernel).
+template <class IO, int N, int KC, int NPT>
+int launch_lag(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st) {
+    using CF = bdk::LagCfg<N, KC, NPT>;
+    using LY = bdk::LagLayout<IO, N, KC, NPT>;
+    auto kern = bdk::bdscan_lag_kernel<IO, N, KC, NPT>;
+    static std::atomic<uint64_t> done_mask{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(done_mask.load(std::memory_order_acquire) & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::bytes);
+        if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
+        done_mask.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    dim3 grid((unsigned)((a.D + bdk::kCh - 1) / bdk::kCh), (unsigned)batch, 1);
+    kern<<<grid, CF::THREADS, LY::bytes, st>>>(a);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
+    return BDSCAN_OK;
+}
+
 template <class IO, int N>
 int dispatch_mode(int mode, const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1,
                   bool thin = false, bool pdl = false) {
@@ -109,6 +132,18 @@ int dispatch_mode(int mode, const bdk::ScanArgs &a, int64_t batch, cudaStream_t 
                 case 32: return launch<IO, N, bdk::kFused, 32, 1>(a, batch, st, 1, pdl);
                 default: return launch<IO, N, bdk::kFused, 0, 1>(a, batch, st, 1, pdl);
             }
+        }
+    }
+    // several whole blocks of 16 or 32 tokens: the lagged schedule (the reverse
+    // chain one block behind the forward chain). Blocks of 4 keep the phased
+    // kernel: their 4-step phases are too short to carry the lag (measured
+    // 8.8 -> 10.2 ms per 350M-stack layer).
+    if (mode == bdk::kFused && !thin && a.L >= 2 * (int64_t)a.K) {
+        if constexpr (N == 16) {
+            if (a.K == 16) return launch_lag<IO, N, 16, 4>(a, batch, st);
+            if (a.K == 32) return launch_lag<IO, N, 32, 4>(a, batch, st);
+        } else {
+            if (a.K == 16) return launch_lag<IO, N, 16, 8>(a, batch, st);
         }
     }
     if constexpr (N == 64) {

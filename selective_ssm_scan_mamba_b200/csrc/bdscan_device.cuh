@@ -171,6 +171,19 @@ __device__ __forceinline__ void tmem_wait_ld(float (&u)[8], float (&v)[8]) {
                  :
                  : "memory");
 }
+__device__ __forceinline__ void tmem_wait_ld(float (&u)[8]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+f"(u[0]), "+f"(u[1]), "+f"(u[2]), "+f"(u[3]), "+f"(u[4]), "+f"(u[5]), "+f"(u[6]), "+f"(u[7])
+                 :
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld(float (&u)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+f"(u[0]), "+f"(u[1]), "+f"(u[2]), "+f"(u[3]), "+f"(u[4]), "+f"(u[5]), "+f"(u[6]), "+f"(u[7]),
+                   "+f"(u[8]), "+f"(u[9]), "+f"(u[10]), "+f"(u[11]), "+f"(u[12]), "+f"(u[13]), "+f"(u[14]), "+f"(u[15])
+                 :
+                 : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld(float (&u)[16], float (&v)[16]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+f"(u[0]), "+f"(u[1]), "+f"(u[2]), "+f"(u[3]), "+f"(u[4]), "+f"(u[5]), "+f"(u[6]), "+f"(u[7]),

@@ -97,7 +97,8 @@ struct Cfg {
     static constexpr int T = (MODE == kFused && (KC == 0 || KC > 16 || (KC == 16 && N == 16))) ? 32
                              : ((MODE == kLongFused && N == 16) ? 32 : 16);   // tokens per tile
     static constexpr int S = T == 16 ? 4 : 3;                                    // cp.async ring depth
-    static constexpr int SPAN = MODE == kFused ? (KC > 0 ? KC : T) : 16;
+    // (forward-only: spans of 8 keep the span's decays and inputs in registers without spills)
+    static constexpr int SPAN = MODE == kFused ? (KC > 0 ? KC : T) : (MODE == kForwardOnly ? 8 : 16);
     static constexpr bool KEEP_B = SPAN <= 16 && N == 16;                        // keep b for phase C
     static constexpr int PER = T / W > 0 ? T / W : 1;                            // readout tokens per warp
     static constexpr int PV = PER >= 4 ? 4 : PER;                                // readout vector width
@@ -653,7 +654,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
             }
         } else if (MODE == kForwardOnly) {
             // forward-only scan (prefill, commit without y, time-chunked pass 2):
-            // (A) decays and inputs of a span, (B) the chain with its readout
+            // (A) decays and inputs of a span of 8, (B) the chain with its readout
             // partials. Full spans (all but a ragged last tile) run without
             // per-token guards; block-end states are tested for only when the
             // caller asked for them.
