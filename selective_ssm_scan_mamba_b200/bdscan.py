@@ -99,26 +99,47 @@ def _need(t, name, dtype, shape, device):
         raise ValueError(f"{name} must be contiguous")
 
 
+_DIMS = {}   # Dims structs by value (read-only once built; the library only reads them during a call)
+
+
+def _dims_of(Bt, L, D, N, K, io, dt_softplus):
+    key = (Bt, L, D, N, K, io, dt_softplus)
+    d = _DIMS.get(key)
+    if d is None:
+        if len(_DIMS) >= 256:
+            _DIMS.clear()
+        d = _DIMS[key] = Dims(*key)
+    return d
+
+
 def _prepare(x, dt, A, B, C_, Dskip, block, z, dt_softplus):
     if not isinstance(x, torch.Tensor) or x.dim() != 3:
         raise ValueError("x must be a [batch, L, D] tensor")
-    _check_device(x.device)
+    dev = x.device
+    _check_device(dev)
     Bt, L, D = x.shape
     N = B.shape[-1] if isinstance(B, torch.Tensor) and B.dim() == 3 else -1
     io = x.dtype
-    if io not in (torch.float32, torch.bfloat16):
+    if io is not torch.float32 and io is not torch.bfloat16:
         raise TypeError("io dtype must be float32 or bfloat16")
-    dev = x.device
-    _need(x, "x", io, (Bt, L, D), dev)
-    _need(dt, "dt", io, (Bt, L, D), dev)
-    _need(B, "B", io, (Bt, L, N), dev)
-    _need(C_, "C", io, (Bt, L, N), dev)
-    _need(A, "A", torch.float32, (D, N), dev)
-    _need(Dskip, "Dskip", torch.float32, (D,), dev)
+    xs, bs, f32 = x.shape, (Bt, L, N), torch.float32
+    # the common path: one pass of cheap tests; the specific error from _need otherwise
+    T = torch.Tensor
+    if not (x.is_contiguous()
+            and isinstance(dt, T) and dt.dtype is io and dt.shape == xs and dt.is_contiguous() and dt.device == dev
+            and isinstance(B, T) and B.dtype is io and B.shape == bs and B.is_contiguous() and B.device == dev
+            and isinstance(C_, T) and C_.dtype is io and C_.shape == bs and C_.is_contiguous() and C_.device == dev
+            and isinstance(A, T) and A.dtype is f32 and A.shape == (D, N) and A.is_contiguous() and A.device == dev
+            and isinstance(Dskip, T) and Dskip.dtype is f32 and Dskip.shape == (D,) and Dskip.is_contiguous()
+            and Dskip.device == dev):
+        for t, name, dtp, shp in ((x, "x", io, (Bt, L, D)), (dt, "dt", io, (Bt, L, D)), (B, "B", io, bs),
+                                  (C_, "C", io, bs), (A, "A", f32, (D, N)), (Dskip, "Dskip", f32, (D,))):
+            _need(t, name, dtp, shp, dev)
     if z is not None:
         _need(z, "z", io, (Bt, L, D), dev)
-    dims = Dims(Bt, L, D, N, int(block), BF16 if io == torch.bfloat16 else F32, 1 if dt_softplus else 0)
-    ins = Inputs(_ptr(x), _ptr(dt), _ptr(B), _ptr(C_), _ptr(z), _ptr(A), _ptr(Dskip))
+    dims = _dims_of(Bt, L, D, N, int(block), BF16 if io is torch.bfloat16 else F32, 1 if dt_softplus else 0)
+    ins = Inputs(x.data_ptr(), dt.data_ptr(), B.data_ptr(), C_.data_ptr(), None if z is None else z.data_ptr(),
+                 A.data_ptr(), Dskip.data_ptr())
     return dims, ins, (Bt, L, D, N), io, dev
 
 
