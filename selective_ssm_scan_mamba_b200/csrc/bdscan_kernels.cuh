@@ -627,10 +627,13 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
                 }
             }
         } else if (MODE == kForwardOnly && chunked && a.chunk_pass == 1) {
-            // time-chunked pass 1: the chunk's state from zero and the product of its decays
+            // time-chunked pass 1: the chunk's state from zero and the product of its
+            // decays (full tiles without per-token branches)
+            auto pass1 = [&](auto whole_tag) {
+                constexpr bool WHOLE = decltype(whole_tag)::value;
 #pragma unroll
             for (int t = 0; t < T; ++t) {
-                if (t < tlen) {
+                if (WHOLE || t < tlen) {
                     float at_[NPT], bq_[NPT];
                     decay_input<NPT>(al, ddc[t * kCh], Bw + t * N, at_, bq_);
                     if constexpr (NPT % 2 == 0) {
@@ -652,15 +655,20 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
                     }
                 }
             }
+            };
+            if (tlen == T) pass1(std::true_type{});
+            else pass1(std::false_type{});
         } else if (MODE == kForwardOnly) {
             // forward-only scan (prefill, commit without y, time-chunked pass 2):
             // (A) decays and inputs of a span of 8, (B) the chain with its readout
             // partials. Full spans (all but a ragged last tile) run without
-            // per-token guards; block-end states are tested for only when the
-            // caller asked for them.
+            // per-token guards, and block-end states are tested for per token
+            // only where a span holds a block end and the caller asked for the
+            // states: every other span is one branch-free basic block, so the
+            // compiler can overlap one token's exps with another's chain.
             const bool wb = endmask != 0 && bnd_ptr != nullptr;
-            auto fwd_span = [&](int s0, auto whole_tag) {
-                constexpr bool WHOLE = decltype(whole_tag)::value;
+            auto fwd_span = [&](int s0, auto whole_tag, auto wb_tag) {
+                constexpr bool WHOLE = decltype(whole_tag)::value, WB = decltype(wb_tag)::value;
                 constexpr int NB = KEEP_B ? SPAN : 1;
                 float at[SPAN][NPT];
                 float bt[NB][NPT];
@@ -685,7 +693,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
                             input_only<NPT>(ddc[t * kCh].y, Bw + t * N, bq);
                         }
                         yp[t] = scan_step<NPT>(h, at[i], bq, Cw + t * N);
-                        if (wb && ((endmask >> t) & 1u)) write_boundary(t0 + t);
+                        if (WB && ((endmask >> t) & 1u)) write_boundary(t0 + t);
                     } else {
                         yp[t] = 0.f;
                     }
@@ -693,8 +701,13 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
             };
 #pragma unroll
             for (int sp = 0; sp < T / SPAN; ++sp) {
-                if (sp * SPAN + SPAN <= tlen) fwd_span(sp * SPAN, std::true_type{});
-                else fwd_span(sp * SPAN, std::false_type{});
+                const bool ends = wb && ((endmask >> (sp * SPAN)) & ((1u << SPAN) - 1u)) != 0;
+                if (sp * SPAN + SPAN <= tlen) {
+                    if (ends) fwd_span(sp * SPAN, std::true_type{}, std::true_type{});
+                    else fwd_span(sp * SPAN, std::true_type{}, std::false_type{});
+                } else {
+                    fwd_span(sp * SPAN, std::false_type{}, std::true_type{});
+                }
             }
         } else {
             // fused with a runtime block length (<= 32)
