@@ -701,7 +701,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
             };
 #pragma unroll
             for (int sp = 0; sp < T / SPAN; ++sp) {
-                const bool ends = wb && ((endmask >> (sp * SPAN)) & ((1u << SPAN) - 1u)) != 0;
+                const bool ends = wb && ((endmask >> (sp * SPAN)) & (SPAN >= 32 ? 0xffffffffu : (1u << (SPAN % 32)) - 1u)) != 0;
                 if (sp * SPAN + SPAN <= tlen) {
                     if (ends) fwd_span(sp * SPAN, std::true_type{}, std::true_type{});
                     else fwd_span(sp * SPAN, std::true_type{}, std::false_type{});
