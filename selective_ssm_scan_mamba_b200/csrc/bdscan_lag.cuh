@@ -22,8 +22,12 @@
 // read from (blocks of even index use slot i for token i, blocks of odd index
 // slot K-1-i). A token's output is complete once both chains have passed it:
 // the forward partial of block j waits in registers for its reverse partial,
-// so the readout of a tile covers the window one block behind it, and a last
-// phase runs the reverse chain of the final block alone.
+// and the sum goes straight to the shared readout buffer (one conflict-free
+// scalar store per step: no register window), so the readout of a tile covers
+// the window one block behind it, and a last phase runs the reverse chain of
+// the final block alone. Tiles are 32 tokens for blocks of 16 and 32 (half the
+// barriers per token of 16-token tiles; one CTA per SM at N = 64 idles the SM
+// at every barrier).
 //
 // Work decomposition as in bdscan_kernel: CTA = 32 channels of one sequence,
 // lane = channel, warp = NPT states; tiles of T tokens (whole blocks) staged by
@@ -38,7 +42,7 @@ namespace bdk {
 template <int N, int KC, int NPTV>
 struct LagCfg {
     static constexpr int K = KC, NPT = NPTV, W = N / NPT, THREADS = 32 * W;
-    static constexpr int T = (K >= 16 && N == 16) ? 32 : 16;   // tokens per tile (whole blocks)
+    static constexpr int T = K >= 16 ? 32 : 16;                // tokens per tile (whole blocks)
     static constexpr int NBT = T / K;                            // blocks per tile
     static constexpr int S = 4;                                  // ring stages, prefetch S - 2 tiles ahead
     static constexpr int TV = 2 * NPT;                           // TMEM columns per token: a, b
@@ -46,7 +50,6 @@ struct LagCfg {
     static constexpr int TNEED = (W / 4) * WCOLS;
     static constexpr int TCOLS = TNEED <= 32 ? 32 : (TNEED <= 64 ? 64 : (TNEED <= 128 ? 128 : (TNEED <= 256 ? 256 : 512)));
     static constexpr int PER = T / W > 0 ? T / W : 1;            // readout tokens per warp
-    static constexpr int PV = PER >= 4 ? 4 : PER;                // readout vector width
     static constexpr int MINB0 = THREADS >= 512 ? 1 : NPT == 8 ? 1 : (K <= 16 ? 3 : 2);
     static constexpr int MINB = 512 / TCOLS < MINB0 ? 512 / TCOLS : MINB0;
     static_assert(W % 4 == 0 && TNEED <= 512 && T % K == 0 && (NPT == 4 || NPT == 8), "lagged layout");
@@ -62,7 +65,7 @@ struct LagLayout {
     static constexpr int dd = S * stage;                   // float2 (delta, delta*x)   [T][32]
     static constexpr int bf = dd + T * kCh * 8;            // float B                  [T][N]
     static constexpr int cf = bf + T * N * 4;              // float C, two tiles       [2][T][N]
-    static constexpr int red = cf + 2 * T * N * 4;         // float partial readouts   [W][T/PV][32][PV]
+    static constexpr int red = cf + 2 * T * N * 4;         // float window partials    [W][T][32]
     static constexpr int bytes = red + W * T * kCh * 4;
     static_assert(xb % 16 == 0 && bb % 16 == 0, "16-byte rows");
 };
@@ -73,7 +76,7 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
     using CF = LagCfg<N, KC, NPTV>;
     using LY = LagLayout<IO, N, KC, NPTV>;
     constexpr int K = CF::K, NPT = CF::NPT, W = CF::W, NT = CF::THREADS, T = CF::T, S = CF::S;
-    constexpr int NBT = CF::NBT, TV = CF::TV, PER = CF::PER, PV = CF::PV;
+    constexpr int NBT = CF::NBT, TV = CF::TV, PER = CF::PER;
 
     extern __shared__ __align__(16) char smem[];
     float2 *dd = reinterpret_cast<float2 *>(smem + LY::dd);
@@ -141,9 +144,7 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
     float yfp[K];   // forward readout partials of the block whose reverse pass comes next
 #pragma unroll
     for (int i = 0; i < K; ++i) yfp[i] = 0.f;
-    float ywin[T];  // complete partials of the readout window (one block behind the tile)
-#pragma unroll
-    for (int i = 0; i < T; ++i) ywin[i] = 0.f;
+    float *redw = red + warp * T * kCh + c;   // this lane's window partials, [W][T][32]
 
     // One phase: the forward chain over block jf (its tokens at local offset bi * K
     // of the current tile) and the reverse chain over block jf - 1.
@@ -184,7 +185,7 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
                 float ar[NPT], br[NPT];
 #pragma unroll
                 for (int q = 0; q < NPT; ++q) { ar[q] = cr[q]; br[q] = cr[NPT + q]; }
-                ywin[bi * K + ir] = __fadd_rn(yfp[ir], scan_step<NPT>(g, ar, br, Cr + (lr0 + ir) * N));
+                redw[(bi * K + ir) * kCh] = __fadd_rn(yfp[ir], scan_step<NPT>(g, ar, br, Cr + (lr0 + ir) * N));
                 if (i + 1 < K) {
                     tmem_wait_ld(nr);
 #pragma unroll
@@ -204,47 +205,14 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
     // before 0 skipped): the W state-group partials of every (token, channel),
     // the skip term, the gate, the store.
     auto readout = [&](int64_t wt0, int nwin) {
-        {
-            float *wrow = red + (warp * (T / PV) * kCh + c) * PV;
-#pragma unroll
-            for (int q = 0; q < T / PV; ++q) {
-                float *dst = wrow + q * kCh * PV;
-                if constexpr (PV == 4)
-                    *reinterpret_cast<float4 *>(dst) =
-                        make_float4(ywin[4 * q], ywin[4 * q + 1], ywin[4 * q + 2], ywin[4 * q + 3]);
-                else if constexpr (PV == 2)
-                    *reinterpret_cast<float2 *>(dst) = make_float2(ywin[2 * q], ywin[2 * q + 1]);
-                else
-                    dst[0] = ywin[q];
-            }
-        }
-        __syncthreads();
+        __syncthreads();   // every warp's window partials are in [W][T][32]
         float ysum[PER];
 #pragma unroll
         for (int i = 0; i < PER; ++i) ysum[i] = 0.f;
 #pragma unroll
         for (int gg = 0; gg < W; ++gg) {
-            const float *rrow = red + ((gg * (T / PV) + warp * (PER / PV)) * kCh + c) * PV;
 #pragma unroll
-            for (int q = 0; q < PER / PV; ++q) {
-                const float *src = rrow + q * kCh * PV;
-                if constexpr (PV == 4) {
-                    const float4 v = *reinterpret_cast<const float4 *>(src);
-                    const float2 s0 = __fadd2_rn(make_float2(ysum[4 * q], ysum[4 * q + 1]), make_float2(v.x, v.y));
-                    const float2 s1 = __fadd2_rn(make_float2(ysum[4 * q + 2], ysum[4 * q + 3]), make_float2(v.z, v.w));
-                    ysum[4 * q] = s0.x;
-                    ysum[4 * q + 1] = s0.y;
-                    ysum[4 * q + 2] = s1.x;
-                    ysum[4 * q + 3] = s1.y;
-                } else if constexpr (PV == 2) {
-                    const float2 v = *reinterpret_cast<const float2 *>(src);
-                    const float2 s0 = __fadd2_rn(make_float2(ysum[2 * q], ysum[2 * q + 1]), v);
-                    ysum[2 * q] = s0.x;
-                    ysum[2 * q + 1] = s0.y;
-                } else {
-                    ysum[q] = __fadd_rn(ysum[q], src[0]);
-                }
-            }
+            for (int i = 0; i < PER; ++i) ysum[i] = __fadd_rn(ysum[i], red[(gg * T + warp * PER + i) * kCh + c]);
         }
         if (want_y && dvalid) {
 #pragma unroll

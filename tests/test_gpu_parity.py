@@ -51,6 +51,9 @@ TRAIN_CASES = [
     (3, 160, 200, 64, 16, "bf16", True, True, True),
     (2, 100, 104, 64, 4, "f32", True, True, True),
     (1, 64, 48, 64, 16, "f32", False, False, False),
+    # an odd number of 16-token blocks: the lagged schedule's last tile is half a tile
+    (1, 112, 40, 64, 16, "bf16", True, True, True),
+    (2, 80, 48, 16, 16, "f32", False, True, True),
     # long blocks whose span checkpoints do not fit in shared memory: the two-sweep path
     (1, 512, 16, 64, 512, "bf16", True, True, True),
     (1, 288, 16, 64, 288, "f32", False, True, True),
