@@ -27,7 +27,10 @@
 // the window one block behind it, and a last phase runs the reverse chain of
 // the final block alone. Tiles are 32 tokens for blocks of 16 and 32 (half the
 // barriers per token of 16-token tiles; one CTA per SM at N = 64 idles the SM
-// at every barrier).
+// at every barrier). The forward chain is software-pipelined by one token: the
+// decay (its exps) and input of token i+1 are formed during step i, so their
+// shared-memory loads and MUFU latency overlap step i's chain work instead of
+// heading the next step.
 //
 // Work decomposition as in bdscan_kernel: CTA = 32 channels of one sequence,
 // lane = channel, warp = NPT states; tiles of T tokens (whole blocks) staged by
@@ -165,6 +168,8 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
         }
         if (F && a.blk_h0) restart_h(jf);
         float yfc[K];
+        float afn[NPT], bqn[NPT];   // decay and input of the next forward token, formed a step ahead
+        if constexpr (F) decay_input<NPT>(al, ddc[bi * K * kCh], Bw + bi * K * N, afn, bqn);
 #pragma unroll
         for (int i = 0; i < K; ++i) {
             float nr[TV];
@@ -174,7 +179,9 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
             if constexpr (F) {
                 const int tl = bi * K + i;
                 float af[NPT], bq[NPT], v[TV];
-                decay_input<NPT>(al, ddc[tl * kCh], Bw + tl * N, af, bq);
+#pragma unroll
+                for (int q = 0; q < NPT; ++q) { af[q] = afn[q]; bq[q] = bqn[q]; }
+                if (i + 1 < K) decay_input<NPT>(al, ddc[(tl + 1) * kCh], Bw + (tl + 1) * N, afn, bqn);
 #pragma unroll
                 for (int q = 0; q < NPT; ++q) { v[q] = af[q]; v[NPT + q] = bq[q]; }
                 tmem_st(tmem_w + slot(jf, i), v);   // the slot block jr's token K-1-i was read from
