@@ -9,7 +9,9 @@ If the library has not been built this module fails to import.
 from __future__ import annotations
 
 import ctypes as ct
+import importlib.util
 import os
+import sysconfig
 
 import torch
 
@@ -67,6 +69,18 @@ _lib.bdscan_last_cuda_error.restype = ct.c_char_p
 
 LIBRARY_PATH = _LIB_PATH
 version = _lib.bdscan_version
+
+# The compiled per-step marshalling module (csrc/bdscan_fastpath.cpp): the same
+# checks and the same C-ABI calls for block_step / commit_block / BlockStep,
+# without the interpreter's per-attribute cost. It answers NOT_COMMON for any
+# case outside the common one, which then takes the checked path below.
+_FAST_PATH = os.path.join(os.path.dirname(_LIB_PATH), "_bdscan_fast" + sysconfig.get_config_var("EXT_SUFFIX"))
+_fast = None
+if os.path.exists(_FAST_PATH):
+    _spec = importlib.util.spec_from_file_location("_bdscan_fast", _FAST_PATH)
+    _fast = importlib.util.module_from_spec(_spec)
+    _spec.loader.exec_module(_fast)
+FASTPATH_LOADED = _fast is not None
 
 
 class BdscanError(RuntimeError):
@@ -338,6 +352,15 @@ def carry_fold(H_all, P_all, index, h0=None, out=None):
 
 def block_step(x, dt, A, B, C, Dskip, h_cache, z=None, dt_softplus=True, y=None):
     """One denoising step of the active block (L == block): returns y. h_cache is read only."""
+    if _fast is not None:
+        try:
+            rc, yo = _fast.block_step(x, dt, A, B, C, Dskip, h_cache, z, bool(dt_softplus), y)
+        except TypeError:   # an argument that is not a tensor: the checked path names it
+            rc = _fast.NOT_COMMON
+        if rc == 0:
+            return yo
+        if rc != _fast.NOT_COMMON:
+            raise BdscanError(rc, "bdscan_block_step")
     block = x.shape[1]
     dims, ins, (Bt, L, D, N), io, dev = _prepare(x, dt, A, B, C, Dskip, block, z, dt_softplus)
     _need(h_cache, "h_cache", torch.float32, (Bt, D, N), dev)
@@ -375,8 +398,19 @@ class BlockStep:
         self._ins = Inputs(None, None, None, None, None, A.data_ptr(), Dskip.data_ptr())
         self._h = h_cache.data_ptr()
         self._dims_ref, self._ins_ref = ct.byref(self._dims), ct.byref(self._ins)
+        self._fast_args = (Bt, K, D, N, dtype == torch.bfloat16, bool(dt_softplus), A.data_ptr(), Dskip.data_ptr(),
+                           self._h)
 
     def __call__(self, x, dt, B, C, y=None, z=None):
+        if _fast is not None and (z is not None) == self.gated:
+            try:
+                rc, yo = _fast.prepared_step(x, dt, B, C, z, y, *self._fast_args)
+            except TypeError:
+                rc = _fast.NOT_COMMON
+            if rc == 0:
+                return yo
+            if rc != _fast.NOT_COMMON:
+                raise BdscanError(rc, "bdscan_block_step")
         xs, bs, io, dev = self.xshape, self.bshape, self.io, self.dev
         for t, name, shp in ((x, "x", xs), (dt, "dt", xs), (B, "B", bs), (C, "C", bs)):
             _need(t, name, io, shp, dev)
@@ -399,6 +433,15 @@ class BlockStep:
 
 def commit_block(x, dt, A, B, C, Dskip, h_cache, z=None, dt_softplus=True, want_y=False, y=None):
     """Commit a clean block (L == block): advances h_cache in place; returns y or None."""
+    if _fast is not None:
+        try:
+            rc, yo = _fast.commit_block(x, dt, A, B, C, Dskip, h_cache, z, bool(dt_softplus), bool(want_y), y)
+        except TypeError:
+            rc = _fast.NOT_COMMON
+        if rc == 0:
+            return yo
+        if rc != _fast.NOT_COMMON:
+            raise BdscanError(rc, "bdscan_commit_block")
     block = x.shape[1]
     dims, ins, (Bt, L, D, N), io, dev = _prepare(x, dt, A, B, C, Dskip, block, z, dt_softplus)
     _need(h_cache, "h_cache", torch.float32, (Bt, D, N), dev)

@@ -158,3 +158,34 @@ def test_prepared_block_step_marshalling(fake):
         gated(t["x"], t["dt"], t["B"], t["C"])
     gated(t["x"], t["dt"], t["B"], t["C"], z=t["x"])
     assert fake.calls[-1][1][1]._obj.z == t["x"].data_ptr()
+
+
+def test_compiled_step_marshalling_declines_other_cases():
+    """The compiled per-step module loads with the binding and links the same
+    library. For anything outside the common case (here: CPU tensors, a
+    non-tensor argument) it answers NOT_COMMON without a library call, and the
+    checked path raises the specific error as before."""
+    assert bdscan.FASTPATH_LOADED
+    f = bdscan._fast
+    t = tensors(L=32)
+    h = torch.zeros(2, 64, 16)
+    rc, y = f.block_step(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], h, None, True, None)
+    assert rc == f.NOT_COMMON and y is None
+    rc, y = f.commit_block(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], h, None, True, True, None)
+    assert rc == f.NOT_COMMON and y is None
+    rc, y = f.prepared_step(t["x"], t["dt"], t["B"], t["C"], None, None, 2, 32, 64, 16, True, True, 0, 0, 0)
+    assert rc == f.NOT_COMMON and y is None
+    with pytest.raises(ValueError, match="CUDA"):
+        bdscan.block_step(t["x"], t["dt"], t["A"], t["B"], t["C"], t["Dskip"], h)
+
+
+def test_non_tensor_argument_reaches_the_checked_path(fake):
+    # the compiled module's argument conversion refuses a list; the checked
+    # path then names the argument
+    t = tensors(L=32)
+    h = torch.zeros(2, 64, 16)
+    with pytest.raises(TypeError, match="Dskip must be a torch.Tensor"):
+        bdscan.block_step(t["x"], t["dt"], t["A"], t["B"], t["C"], [0.0], h)
+    with pytest.raises(TypeError, match="Dskip must be a torch.Tensor"):
+        bdscan.commit_block(t["x"], t["dt"], t["A"], t["B"], t["C"], [0.0], h)
+    assert fake.calls == []
