@@ -20,7 +20,11 @@
 //            8 tokens (K <= 8) or one block (K > 8). The forward state at a
 //            segment start is the forward pass's block-boundary state (h0 for
 //            the first), so no forward state is stored by the forward pass
-//            beyond the caches it writes anyway.
+//            beyond the caches it writes anyway. At N = 16 that state is copied
+//            into the ring stage of the segment's first tile with the tile's
+//            inputs (cp.async, two steps ahead), so no tile waits on a global
+//            load of it; at N = 64 the dB | dC tile leaves no room and it is
+//            loaded directly.
 //   long   = for K > 8 the block's tiles are first swept forwards (phase 1) to
 //            leave (h, a_t mu_t) checkpoints at tile starts in the workspace;
 //            the tiles then run last to first (phase 2).
@@ -82,7 +86,11 @@ struct BwdLayout {
     static constexpr int TT = CF::TT, W = CF::W;
     static constexpr int xb = TT * kCh * (int)sizeof(IO);   // one x / dt / z / dy tile
     static constexpr int bb = TT * N * (int)sizeof(IO);     // one B / C tile
-    static constexpr int stage = 4 * xb + 2 * bb;
+    // the segment's start state [W][32][4], staged with a segment's first tile
+    // (N = 16 only: at N = 64 the dB | dC tile leaves no room for it)
+    static constexpr bool HS = N == 16;
+    static constexpr int hs = 4 * xb + 2 * bb;
+    static constexpr int stage = hs + (HS ? W * kCh * 16 : 0);
     static constexpr int dq = CF::S * stage;                // float4 (delta, delta*x, ds, d delta/d dt) [TT][32]
     static constexpr int bf = dq + TT * kCh * 16;           // float B  [TT][N]
     static constexpr int cf = bf + TT * N * 4;              // float C  [TT][N]
@@ -221,20 +229,31 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
         if (iq >= 0) {
             const BwdTile tl = bwd_tile(iq, ir, ntb, SL, L, longb, TT);
             stage_bwd_tile<IO, N, TT, NT>(smem + slot * LY::stage, a, b, d0, tl.t0, tl.tlen, gated);
+            if (LY::HS && tl.i == 0) {   // the forward state at the segment start, staged with its first tile
+                const float *src = tl.ts == 0 ? (a.h0 ? a.h0 + (b * a.D + d) * N + n0 : nullptr)
+                                              : a.boundary + ((b * nblk + tl.ts / K - 1) * a.D + d) * N + n0;
+                const bool ok = dvalid && src != nullptr;
+                cp_async16(smem + slot * LY::stage + LY::hs + tid * 16, ok ? static_cast<const void *>(src) : a.x, ok);
+            }
             advance(iq, ir);
         }
         cp_async_commit();
     };
     float *ck_base = a.ws_ck ? a.ws_ck + (((b * CT + ct) * a.nck * W + warp) * kCh + c) * 8 : nullptr;
     const int64_t ck_stride = (int64_t)W * kCh * 8;   // between consecutive checkpoints of this lane
-    auto init_segment = [&](int64_t ts) {   // forward state at a block start, reverse adjoint zero
-        const float *src = ts == 0 ? (a.h0 ? a.h0 + (b * a.D + d) * N + n0 : nullptr)
-                                   : a.boundary + ((b * nblk + ts / K - 1) * a.D + d) * N + n0;
+    auto init_segment = [&](const char *st, int64_t ts) {   // forward state at a block start, reverse adjoint zero
+        if constexpr (LY::HS) {
+            const float4 hv = *reinterpret_cast<const float4 *>(st + LY::hs + tid * 16);
+            h2[0] = make_float2(hv.x, hv.y);
+            h2[1] = make_float2(hv.z, hv.w);
+        } else {
+            const float *src = ts == 0 ? (a.h0 ? a.h0 + (b * a.D + d) * N + n0 : nullptr)
+                                       : a.boundary + ((b * nblk + ts / K - 1) * a.D + d) * N + n0;
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            h2[p] = (dvalid && src) ? make_float2(src[2 * p], src[2 * p + 1]) : f2(0.f);
-            nu2[p] = f2(0.f);
+            for (int p = 0; p < 2; ++p) h2[p] = (dvalid && src) ? make_float2(src[2 * p], src[2 * p + 1]) : f2(0.f);
         }
+        nu2[0] = f2(0.f);
+        nu2[1] = f2(0.f);
     };
 
     const float4 *dqc = dq + c;
@@ -293,7 +312,7 @@ __global__ void __launch_bounds__(BwdCfg<N>::THREADS, BwdCfg<N>::MINB) bdscan_bw
 
         // ---- state at the tile start -------------------------------------------
         if (tl.i == 0) {
-            init_segment(tl.ts);
+            init_segment(st, tl.ts);
         } else if (!tl.ph1 && tl.i < ntb - 1) {   // (tile ntb-1 continues from phase 1's registers)
             const float4 hv = *reinterpret_cast<const float4 *>(ck_base + (tl.i - 1) * ck_stride);
             const float4 nv = *reinterpret_cast<const float4 *>(ck_base + (tl.i - 1) * ck_stride + 4);
