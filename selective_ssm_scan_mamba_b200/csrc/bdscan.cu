@@ -6,6 +6,7 @@
 
 #include "../../include/bdscan.h"
 #include "bdscan_backward.cuh"
+#include "bdscan_backward16.cuh"
 #include "bdscan_kernels.cuh"
 #include "bdscan_lag.cuh"
 
@@ -372,18 +373,21 @@ int launch_bwd(const bdk::BwdArgs &a, int64_t batch, int64_t ct, void *dB, void 
                cudaStream_t st) {
     using CF = bdk::BwdCfg<N>;
     using LY = bdk::BwdLayout<IO, N>;
-    auto kern = bdk::bdscan_bwd_kernel<IO, N>;
+    // blocks of 16 at N = 16: each block staged once (bdscan_bwd16_kernel)
+    const bool b16 = N == 16 && a.K == 16;
+    auto kern = b16 ? bdk::bdscan_bwd16_kernel<IO> : bdk::bdscan_bwd_kernel<IO, N>;
+    const int smem = b16 ? bdk::Bwd16Layout<IO>::bytes : LY::bytes;
     static std::atomic<uint64_t> done_mask{0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
-    const uint64_t bit = 1ull << (dev & 63);
+    const uint64_t bit = 1ull << ((2 * dev + (b16 ? 1 : 0)) & 63);
     if (!(done_mask.load(std::memory_order_acquire) & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::bytes);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
         done_mask.fetch_or(bit, std::memory_order_acq_rel);
     }
     if (batch > 0 && ct > 0) {
-        kern<<<dim3((unsigned)ct, (unsigned)batch), CF::THREADS, LY::bytes, st>>>(a);
+        kern<<<dim3((unsigned)ct, (unsigned)batch), CF::THREADS, smem, st>>>(a);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
     }

@@ -73,6 +73,10 @@ CASES = [
     (1, 70, 24, 64, 7, "f32", False, True, True),
     (1, 40, 32, 16, 8, "f32", True, True, True),
     (1, 24, 32, 16, 24, "f32", True, True, True),
+    # blocks of 16 at N = 16 (each block staged once): one block with a ragged
+    # channel tile and no softplus, and ten gated blocks over three channel tiles
+    (1, 16, 40, 16, 16, "bf16", False, True, False),
+    (3, 160, 96, 16, 16, "f32", True, True, True),
 ]
 
 
