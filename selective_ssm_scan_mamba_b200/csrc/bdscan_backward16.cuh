@@ -29,8 +29,10 @@
 // per-token guard and the block-start / block-end resets are fixed: the
 // reverse state g is zero after token 15, the reverse adjoint a*mu is zero
 // before token 0. The ring has two stages (the next block is copied while this
-// one is processed). The arithmetic per token is that of bdscan_bwd_kernel,
-// operation for operation, so both kernels give the same bits.
+// one is processed). The readout's P and Q partials share one float2 per
+// (token, channel) (half the shared-memory loads of the readout). The
+// arithmetic per token and every summation order are those of
+// bdscan_bwd_kernel, so both kernels give the same bits.
 #pragma once
 
 #include "bdscan_backward.cuh"
@@ -48,7 +50,7 @@ struct Bwd16Layout {
     static constexpr int dq = S * stage;                    // float4 (delta, delta*x, ds, d delta/d dt) [16][32]
     static constexpr int bf = dq + TB * kCh * 16;           // float B  [16][N]
     static constexpr int cf = bf + TB * N * 4;              // float C  [16][N]
-    static constexpr int red = cf + TB * N * 4;             // float [3][W][8][32]: P, Q, S partials of a half
+    static constexpr int red = cf + TB * N * 4;             // float2 [W][8][32] (P, Q) + float [W][8][32] S partials of a half
     static constexpr int bc = red + 3 * W * TT * kCh * 4;   // float [8][32][BR]: per-lane dB | dC terms of a half
     static constexpr int dsk = bc + TT * kCh * BR * 4;      // float [W][32]: dDskip partials
     static constexpr int bytes = dsk + W * kCh * 4;
@@ -118,7 +120,8 @@ __global__ void __launch_bounds__(128, 3) bdscan_bwd16_kernel(const BwdArgs a) {
     const float4 *dqc = dq + c;
     const float *Bw = Bf + n0;
     const float *Cw = Cf + n0;
-    float *redw = red + (warp * TT) * kCh + c;   // [q][warp][t][lane]
+    float2 *redpq = reinterpret_cast<float2 *>(red) + (warp * TT) * kCh + c;   // [warp][t][lane]
+    float *reds = red + 2 * W * TT * kCh + (warp * TT) * kCh + c;                 // [warp][t][lane]
 
     // forward sweep over the 8 tokens at dqc / Bw / Cw (STORE: into TMEM for the backward sweep)
     auto fwd_sweep = [&](auto store_tag) {
@@ -196,9 +199,8 @@ __global__ void __launch_bounds__(128, 3) bdscan_bwd16_kernel(const BwdArgs a) {
                 rho2[p] = __fmul2_rn(a2, lam2);
                 g2[p] = gn2;
             }
-            redw[t * kCh] = __fadd_rn(P2.x, P2.y);
-            redw[(W * TT + t) * kCh] = __fadd_rn(Q2.x, Q2.y);
-            if (GATED) redw[(2 * W * TT + t) * kCh] = __fadd_rn(S2.x, S2.y);
+            redpq[t * kCh] = make_float2(__fadd_rn(P2.x, P2.y), __fadd_rn(Q2.x, Q2.y));
+            if (GATED) reds[t * kCh] = __fadd_rn(S2.x, S2.y);
             float *brow = bcr + (t * kCh + c) * BR + n0;
             *reinterpret_cast<float4 *>(brow) = make_float4(dB2[0].x, dB2[0].y, dB2[1].x, dB2[1].y);
             *reinterpret_cast<float4 *>(brow + N) = make_float4(dC2[0].x, dC2[0].y, dC2[1].x, dC2[1].y);
@@ -223,10 +225,10 @@ __global__ void __launch_bounds__(128, 3) bdscan_bwd16_kernel(const BwdArgs a) {
                 float P = 0.f, Q = 0.f, Sg = 0.f;
 #pragma unroll
                 for (int gg = 0; gg < W; ++gg) {
-                    const float *rr = red + (gg * TT + t) * kCh + c;
-                    P = __fadd_rn(P, rr[0]);
-                    Q = __fadd_rn(Q, rr[W * TT * kCh]);
-                    if (gated) Sg = __fadd_rn(Sg, rr[2 * W * TT * kCh]);
+                    const float2 pq = reinterpret_cast<const float2 *>(red)[(gg * TT + t) * kCh + c];
+                    P = __fadd_rn(P, pq.x);
+                    Q = __fadd_rn(Q, pq.y);
+                    if (gated) Sg = __fadd_rn(Sg, red[2 * W * TT * kCh + (gg * TT + t) * kCh + c]);
                 }
                 const int e = t * kCh + c;
                 const float4 q4 = dq[r0 * kCh + e];
