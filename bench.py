@@ -393,7 +393,7 @@ def run_ours(args):
     elem = w.batch * w.L * w.D * w.N
     nbytes = algorithmic_bytes(w, boundary=False, h_out=False)
     roof = roofline(elem, nbytes, launch_ms, peaks, traffic_for("stack350m"),
-                    kernel=f"bdscan_kernel<bf16, N=64, fused, K={K}>")
+                    kernel=f"bdscan_lag_kernel<bf16, N=64, K={K}, 8 states per lane>")
 
     # the other block sizes of the stack (same inputs, 24 layers each)
     by_block = {str(K): {"ms_24_layers": ms_per_step, "tokens_per_s": value / world, "sfu_frac": roof["frac"],
@@ -543,7 +543,7 @@ def measure_train(dev, peaks, steps=20, warmup=5) -> dict:
                        "io_dtype": w.io, "outputs": "y + all block-boundary states + final state"},
             "ms": ms, "tokens_per_s": w.batch * w.L / (ms * 1e-3),
             "roofline": roofline(w.batch * w.L * w.D * w.N, algorithmic_bytes(w), ms, peaks, traffic_for("train"),
-                                 kernel="bdscan_kernel<bf16, N=16, fused, K=16>")}
+                                 kernel="bdscan_lag_kernel<bf16, N=16, K=16, 4 states per lane>")}
 
 
 # ------------------------------------------------------- inference workloads

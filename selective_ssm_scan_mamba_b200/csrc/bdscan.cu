@@ -9,6 +9,7 @@
 #include "bdscan_backward16.cuh"
 #include "bdscan_kernels.cuh"
 #include "bdscan_lag.cuh"
+#include "bdscan_step.cuh"
 
 namespace {
 
@@ -122,16 +123,53 @@ int launch_lag(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st) {
     return BDSCAN_OK;
 }
 
+// A block step (or a commit with y) of few rows at N = 16 (bdscan_step_kernel).
+template <class IO, int KC>
+int launch_step(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, bool pdl) {
+    constexpr int T = KC > 0 ? KC : 32;
+    constexpr int smem = bdk::StepLayout<IO, T>::bytes;
+    auto kern = bdk::bdscan_step_kernel<IO, KC>;
+    static std::atomic<uint64_t> done_mask{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(done_mask.load(std::memory_order_acquire) & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
+        done_mask.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    dim3 grid((unsigned)((a.D + bdk::kCh - 1) / bdk::kCh), (unsigned)batch, 1);
+    if (pdl) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(bdk::kStepThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, a);
+        if (le != cudaSuccess) { (void)cudaGetLastError(); g_last_cuda = le; return BDSCAN_ERR_CUDA; }
+    } else {
+        kern<<<grid, bdk::kStepThreads, smem, st>>>(a);
+    }
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
+    return BDSCAN_OK;
+}
+
 template <class IO, int N>
 int dispatch_mode(int mode, const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1,
                   bool thin = false, bool pdl = false) {
     if constexpr (N == 16) {
         if (thin && mode == bdk::kFused) {   // one state per lane: the latency-bound small block step
             switch (a.K) {
-                case 4: return launch<IO, N, bdk::kFused, 4, 1>(a, batch, st, 1, pdl);
-                case 16: return launch<IO, N, bdk::kFused, 16, 1>(a, batch, st, 1, pdl);
-                case 32: return launch<IO, N, bdk::kFused, 32, 1>(a, batch, st, 1, pdl);
-                default: return launch<IO, N, bdk::kFused, 0, 1>(a, batch, st, 1, pdl);
+                case 4: return launch_step<IO, 4>(a, batch, st, pdl);
+                case 16: return launch_step<IO, 16>(a, batch, st, pdl);
+                case 32: return launch_step<IO, 32>(a, batch, st, pdl);
+                default: return launch_step<IO, 0>(a, batch, st, pdl);
             }
         }
     }
@@ -243,7 +281,8 @@ int run(Op op, const bdscan_dims *dm, const bdscan_inputs *in, const float *h0, 
     const unsigned gz = ch ? (unsigned)ch->count : 1u;
     a.L = dm->seqlen; a.D = dm->d_inner; a.K = (int32_t)dm->block; a.dt_softplus = dm->dt_softplus;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // a block step (or a commit with y) over at most one CTA per SM runs thin
+    // a block step (or a commit with y) of at most one (batch, 32-channel) row
+    // per SM runs bdscan_step_kernel (one state per lane)
     bool thin = false;
     if ((op == kStep || (op == kCommit && y)) && mode == bdk::kFused && dm->d_state == 16)
         thin = dm->batch * ((dm->d_inner + bdk::kCh - 1) / bdk::kCh) <= device_sm_count();

@@ -84,11 +84,9 @@ struct ScanArgs {
 // NPT = states per lane: 4 (one warp per 4 states) by default; 8 for the
 // whole-block fused variants at N = 64 (8 warps per CTA: half the per-element
 // shared-memory reads of delta and of the readout partials, twice the
-// independent work per warp); 1 for the thin block-step variant (16 warps per
-// CTA at N = 16), which a block step of too few channels to fill the GPU uses:
-// its 32 tokens are a latency chain, and a quarter of the per-token work per
-// warp shortens it. Prefills of too few channels get their parallelism from
-// time chunks (bdscan_prefill_chunked) instead.
+// independent work per warp). A block step of too few channels to fill the GPU
+// runs bdscan_step_kernel (one state per lane) instead, and prefills of too few
+// channels get their parallelism from time chunks (bdscan_prefill_chunked).
 template <int N, int MODE, int KC, int NPTV = 4>
 struct Cfg {
     static constexpr int NPT = NPTV;
@@ -141,7 +139,7 @@ struct Layout {
     static_assert(xb % 16 == 0 && bb % 16 == 0, "16-byte rows");
 };
 
-// ---- per-lane arithmetic on NPT states (NPT = 1, 2 or 4) -----------------------
+// ---- per-lane arithmetic on NPT states (NPT = 1, 2, 4 or 8) -------------------
 // Every mode runs these same instructions, so the forward state is
 // bit-identical whichever kernel variant computes it (packed and scalar fp32
 // operations round identically).
