@@ -138,8 +138,9 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
 #pragma unroll
         for (int q = 0; q < NPT; ++q) h[q] = (dvalid && src) ? src[q] : 0.f;
     };
-    // TMEM slot of token i of block j
-    auto slot = [](int64_t j, int i) -> uint32_t { return (uint32_t)((j & 1) ? K - 1 - i : i) * TV; };
+    // TMEM slot of token i of a block: slot i in blocks of even index, K-1-i in
+    // blocks of odd index
+    auto slot = [](bool odd, int i) -> uint32_t { return (uint32_t)(odd ? K - 1 - i : i) * TV; };
 
     const float2 *ddc = dd + c;
     const float *Bw = Bf + n0;
@@ -150,9 +151,12 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
     float *redw = red + warp * T * kCh + c;   // this lane's window partials, [W][T][32]
 
     // One phase: the forward chain over block jf (its tokens at local offset bi * K
-    // of the current tile) and the reverse chain over block jf - 1.
-    auto phase = [&](int bi, int64_t jf, int64_t cur_tile, auto f_tag, auto r_tag) {
+    // of the current tile) and the reverse chain over block jf - 1. par_tag: the
+    // parity of jf when it is known at compile time (0 or 1), else -1.
+    auto phase = [&](int bi, int64_t jf, int64_t cur_tile, auto f_tag, auto r_tag, auto par_tag) {
         constexpr bool F = decltype(f_tag)::value, R = decltype(r_tag)::value;
+        constexpr int PAR = decltype(par_tag)::value;
+        const bool fodd = PAR >= 0 ? PAR == 1 : (jf & 1) != 0;   // block jf odd (block jr = jf - 1 even)
         const int64_t jr = jf - 1;
         const float *Cc = Cf2 + (cur_tile & 1) * T * N + n0;                    // C of the current tile
         const int64_t rtile = R ? (jr * K) / T : 0;
@@ -163,7 +167,7 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
         for (int q = 0; q < NPT; ++q) g[q] = 0.f;
         float cr[TV];
         if constexpr (R) {
-            tmem_ld(tmem_w + slot(jr, K - 1), cr);
+            tmem_ld(tmem_w + slot(!fodd, K - 1), cr);
             tmem_wait_ld(cr);
         }
         if (F && a.blk_h0) restart_h(jf);
@@ -174,7 +178,7 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
         for (int i = 0; i < K; ++i) {
             float nr[TV];
             if constexpr (R) {
-                if (i + 1 < K) tmem_ld(tmem_w + slot(jr, K - 2 - i), nr);   // the next reverse token
+                if (i + 1 < K) tmem_ld(tmem_w + slot(!fodd, K - 2 - i), nr);   // the next reverse token
             }
             if constexpr (F) {
                 const int tl = bi * K + i;
@@ -184,7 +188,7 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
                 if (i + 1 < K) decay_input<NPT>(al, ddc[(tl + 1) * kCh], Bw + (tl + 1) * N, afn, bqn);
 #pragma unroll
                 for (int q = 0; q < NPT; ++q) { v[q] = af[q]; v[NPT + q] = bq[q]; }
-                tmem_st(tmem_w + slot(jf, i), v);   // the slot block jr's token K-1-i was read from
+                tmem_st(tmem_w + slot(fodd, i), v);   // the slot block jr's token K-1-i was read from
                 yfc[i] = scan_step<NPT>(h, af, bq, Cc + tl * N);
             }
             if constexpr (R) {
@@ -210,7 +214,10 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
 
     // Readout of nwin window tokens starting at absolute token wt0 (tokens
     // before 0 skipped): the W state-group partials of every (token, channel),
-    // the skip term, the gate, the store.
+    // the skip term, the gate, the store. Warp w finishes window tokens
+    // [w PER, (w+1) PER): wt0 and nwin are multiples of K, and K and T of PER,
+    // so a warp's tokens lie in one tile and are all in the window or all out.
+    static_assert(K % PER == 0 && T % PER == 0, "a warp's readout tokens share a tile");
     auto readout = [&](int64_t wt0, int nwin) {
         __syncthreads();   // every warp's window partials are in [W][T][32]
         float ysum[PER];
@@ -221,22 +228,21 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
 #pragma unroll
             for (int i = 0; i < PER; ++i) ysum[i] = __fadd_rn(ysum[i], red[(gg * T + warp * PER + i) * kCh + c]);
         }
-        if (want_y && dvalid) {
+        const int tw0 = warp * PER;
+        const int64_t ta0 = wt0 + tw0;
+        if (want_y && dvalid && tw0 < nwin && ta0 >= 0) {
+            const int64_t tile = ta0 / T;   // the tokens' staging stage is still in the ring
+            const int lt0 = (int)(ta0 - tile * T);
+            const IO *xs = reinterpret_cast<const IO *>(smem + (int)(tile % S) * LY::stage) + lt0 * kCh + c;
+            const IO *zs = xs + 2 * T * kCh;
+            IO *yo = static_cast<IO *>(a.y) + (b * L + ta0) * a.D + d;
 #pragma unroll
             for (int i = 0; i < PER; ++i) {
-                const int tw = warp * PER + i;
-                const int64_t ta = wt0 + tw;
-                if (tw < nwin && ta >= 0) {
-                    const int64_t tile = ta / T;   // the token's staging stage is still in the ring
-                    const int lt = (int)(ta - tile * T);
-                    const IO *xs = reinterpret_cast<const IO *>(smem + (tile % S) * LY::stage);
-                    const IO *zs = xs + 2 * T * kCh;
-                    float v = __fmaf_rn(dfac, to_f32(xs[lt * kCh + c]), ysum[i]);
-                    if (gated) v = __fmul_rn(v, silu_f32(to_f32(zs[lt * kCh + c])));
-                    IO o;
-                    from_f32(v, o);
-                    static_cast<IO *>(a.y)[(b * L + ta) * a.D + d] = o;
-                }
+                float v = __fmaf_rn(dfac, to_f32(xs[i * kCh]), ysum[i]);
+                if (gated) v = __fmul_rn(v, silu_f32(to_f32(zs[i * kCh])));
+                IO o;
+                from_f32(v, o);
+                yo[i * a.D] = o;
             }
         }
     };
@@ -273,18 +279,29 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
         __syncthreads();
         const int nb = tlen / K;   // blocks of this tile
         const int64_t b0 = s * NBT;
+        using PEven = std::integral_constant<int, 0>;
+        using POdd = std::integral_constant<int, 1>;
+        using PRun = std::integral_constant<int, -1>;
+        if constexpr (NBT == 2) {   // b0 is even: block b0 + bi has the parity of bi
+            if (nb > 0) {
+                if (s == 0) phase(0, b0, s, std::true_type{}, std::false_type{}, PEven{});
+                else phase(0, b0, s, std::true_type{}, std::true_type{}, PEven{});
+            }
+            if (nb > 1) phase(1, b0 + 1, s, std::true_type{}, std::true_type{}, POdd{});
+        } else {
 #pragma unroll
-        for (int bi = 0; bi < NBT; ++bi) {
-            if (bi < nb) {
-                if (bi == 0 && s == 0) phase(bi, b0 + bi, s, std::true_type{}, std::false_type{});
-                else phase(bi, b0 + bi, s, std::true_type{}, std::true_type{});
+            for (int bi = 0; bi < NBT; ++bi) {
+                if (bi < nb) {
+                    if (bi == 0 && s == 0) phase(bi, b0 + bi, s, std::true_type{}, std::false_type{}, PRun{});
+                    else phase(bi, b0 + bi, s, std::true_type{}, std::true_type{}, PRun{});
+                }
             }
         }
         readout((b0 - 1) * K, nb * K);
     }
     if (nblk > 0) {   // the reverse chain of the last block, then its readout
         __syncthreads();   // every warp is past the last tile's readout of the shared partials
-        phase(0, nblk, nt, std::false_type{}, std::true_type{});
+        phase(0, nblk, nt, std::false_type{}, std::true_type{}, std::integral_constant<int, -1>{});
         readout((nblk - 1) * K, K);
     }
     cp_async_wait<0>();
