@@ -264,6 +264,7 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
             const IO *Bs = dts + 2 * T * kCh;
             const IO *Cs = Bs + T * N;
             float *Cc = Cf2 + (s & 1) * T * N;
+#pragma unroll
             for (int e = tid; e < T * kCh; e += NT) {
                 const float xv = to_f32(xs[e]);
                 const float dr = to_f32(dts[e]);
@@ -271,6 +272,7 @@ __global__ void __launch_bounds__(LagCfg<N, KC, NPTV>::THREADS, LagCfg<N, KC, NP
                 dd[e] = make_float2(dl, __fmul_rn(dl, xv));
             }
             constexpr int EPC = 16 / (int)sizeof(IO);
+#pragma unroll
             for (int e = tid; e < T * N / EPC; e += NT) {
                 widen16(Bs + e * EPC, Bf + e * EPC);
                 widen16(Cs + e * EPC, Cc + e * EPC);
