@@ -433,6 +433,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
         {
             const IO *Bs = zs + T * kCh;
             const IO *Cs = Bs + T * N;
+#pragma unroll
             for (int e = tid; e < T * kCh; e += NT) {
                 const float xv = to_f32(xs[e]);
                 const float dr = to_f32(dts[e]);
@@ -441,6 +442,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
                 dd[e] = make_float2(dl, __fmul_rn(dl, xv));
             }
             constexpr int EPC = 16 / (int)sizeof(IO);
+#pragma unroll
             for (int e = tid; e < T * N / EPC; e += NT) {
                 widen16(Bs + e * EPC, Bf + e * EPC);
                 widen16(Cs + e * EPC, Cf + e * EPC);
@@ -821,7 +823,8 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
                     }
                 }
             }
-            IO *gy = want_y ? static_cast<IO *>(a.y) + (b * L + t0) * a.D + d : nullptr;
+            // this warp's first token of the tile; y rows advance by D per token
+            IO *gy = want_y ? static_cast<IO *>(a.y) + (b * L + t0 + warp * PER) * a.D + d : nullptr;
 #pragma unroll
             for (int i = 0; i < PER; ++i) {
                 const int t = warp * PER + i;
@@ -829,12 +832,12 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
                     const int yr = (int)(t0 - (t0 / K) * K) + t;   // token within its block (long path)
                     if (MODE == kReverseAcc) {
                         if (want_y && dvalid) {   // y holds y_fwd + Dskip x from the forward pass
-                            float v = __fadd_rn(to_f32(gy[(int64_t)t * a.D]), ysum[i]);
+                            float v = __fadd_rn(to_f32(gy[(int64_t)i * a.D]), ysum[i]);
                             v = __fmaf_rn(dskip, to_f32(xs[t * kCh + c]), v);
                             if (gated) v = __fmul_rn(v, silu_f32(to_f32(zs[t * kCh + c])));
                             IO o;
                             from_f32(v, o);
-                            gy[(int64_t)t * a.D] = o;
+                            gy[(int64_t)i * a.D] = o;
                         }
                     } else if (MODE == kLong && rev) {
                         yrev[yr * kCh + c] = ysum[i];
@@ -845,7 +848,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
                         if (gated) v = __fmul_rn(v, silu_f32(to_f32(zs[t * kCh + c])));
                         IO o;
                         from_f32(v, o);
-                        gy[(int64_t)t * a.D] = o;
+                        gy[(int64_t)i * a.D] = o;
                     }
                 }
             }
