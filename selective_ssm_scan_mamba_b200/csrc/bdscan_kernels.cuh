@@ -340,10 +340,23 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
                                               : (tend - tbeg + TE - 1) / TE;   // kReverseAcc: TE = T
     const int nspan = MODE == kLongFused ? (int)((K + SPAN - 1) / SPAN) : 1;   // spans per block
     int64_t tile_in_blk = 0;   // long modes: index of the current tile inside its block
-    auto tile_of = [&](int64_t s, int64_t &t0, int &tlen, bool &rev, bool &first_rev) {
+    // long modes: step s is step r of block j (s = j * per + r), tracked by
+    // cursors that advance one step at a time (no division per step)
+    const int per = (int)(MODE == kLongFused ? nr_blk + nt_blk : 2 * nt_blk);
+    struct Cursor {
+        int64_t j;
+        int r;
+    };
+    auto advance = [&](Cursor &cu) {
+        if (++cu.r == per) {
+            cu.r = 0;
+            ++cu.j;
+        }
+    };
+    auto tile_of = [&](int64_t s, const Cursor &cu, int64_t &t0, int &tlen, bool &rev, bool &first_rev) {
         if (MODE == kLongFused) {
-            const int per = (int)(nr_blk + nt_blk);
-            const int j = (int)s / per, r = (int)s - j * per;   // 32-bit: steps < 2^31
+            const int64_t j = cu.j;
+            const int r = cu.r;
             rev = r < nr_blk;
             const int64_t i = rev ? nt_blk - 1 - r : r - nr_blk;
             first_rev = rev && r == 0;
@@ -352,7 +365,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
             const int64_t rem = (j + 1) * K - t0;
             tlen = (int)(rem < T ? rem : T);
         } else if (MODE == kLong) {
-            const int64_t j = s / (2 * nt_blk), r = s % (2 * nt_blk);
+            const int64_t j = cu.j, r = cu.r;
             rev = r < nt_blk;
             const int64_t i = rev ? nt_blk - 1 - r : r - nt_blk;
             first_rev = rev && r == 0;
@@ -374,15 +387,17 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
             tlen = (int)(rem < TE ? rem : TE);
         }
     };
+    Cursor cur{0, 0}, icur{0, 0};   // the loop's step and the next step to stage (issue() runs in step order)
     auto issue = [&](int64_t s) {
         if (s < nsteps) {
             int64_t t0; int tlen; bool rv, fr;
-            tile_of(s, t0, tlen, rv, fr);
+            tile_of(s, icur, t0, tlen, rv, fr);
             // the g-only reverse sweep and the chunk-summary pass read no C, z
             const bool state_only = (MODE == kLongFused && rv) || (MODE == kForwardOnly && a.chunk_pass == 1);
             stage_tile<IO, N, T, NT>(smem + (s % S) * LY::stage, a, b, d0, t0, tlen, gated && !state_only,
                                      !state_only);
         }
+        advance(icur);
         cp_async_commit();
     };
 
@@ -419,7 +434,8 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
 #pragma unroll 1
     for (int64_t s = 0; s < nsteps; ++s) {
         int64_t t0; int tlen; bool rev, first_rev;
-        tile_of(s, t0, tlen, rev, first_rev);
+        tile_of(s, cur, t0, tlen, rev, first_rev);
+        advance(cur);
         const int64_t ti = tile_in_blk;   // (issue() below reuses tile_of)
         cp_async_wait<S - 2>();
         __syncthreads();   // stage s landed for every thread; step s-1 is fully done
