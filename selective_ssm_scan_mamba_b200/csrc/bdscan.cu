@@ -52,6 +52,8 @@ size_t long_fused_ck_bytes(int64_t K, int N) {
     return (size_t)(spans - 1) * (size_t)N * bdk::kCh * 4;
 }
 
+// (measured on the 4-states-per-lane layout, the larger one: the 8-state kernel
+// that runs at N = 64 takes the same blocks)
 template <class IO, int N>
 bool long_fused_fits(int64_t K) {
     return bdk::Layout<IO, N, bdk::kLongFused, 0>::base_bytes + long_fused_ck_bytes(K, N) <= (size_t)kMaxDynSmem;
@@ -193,7 +195,12 @@ int dispatch_mode(int mode, const bdk::ScanArgs &a, int64_t batch, cudaStream_t 
     }
     if (mode == bdk::kForwardOnly) return launch<IO, N, bdk::kForwardOnly, 0>(a, batch, st, gz, pdl);
     if (mode == bdk::kLong) return launch<IO, N, bdk::kLong, 0>(a, batch, st, 1, pdl);
-    if (mode == bdk::kLongFused) return launch<IO, N, bdk::kLongFused, 0>(a, batch, st, 1, pdl);
+    if (mode == bdk::kLongFused) {
+        if constexpr (N == 64)   // 8 states per lane: a span's a, b fill the SM's TMEM
+            return launch<IO, N, bdk::kLongFused, 0, 8>(a, batch, st, 1, pdl);
+        else
+            return launch<IO, N, bdk::kLongFused, 0>(a, batch, st, 1, pdl);
+    }
     if (mode == bdk::kReverseAcc) return launch<IO, N, bdk::kReverseAcc, 0>(a, batch, st, 1, pdl);
     switch (a.K) {
         case 4: return launch<IO, N, bdk::kFused, 4>(a, batch, st, 1, pdl);

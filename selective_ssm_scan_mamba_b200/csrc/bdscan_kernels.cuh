@@ -109,7 +109,7 @@ struct Cfg {
     static constexpr int WCOLS = SPAN * 2 * NPT;
     static constexpr int TNEED = (W / 4) * WCOLS;
     static constexpr bool TMEM = ((MODE == kFused && KC > 0) || MODE == kLongFused) && W % 4 == 0 &&
-                                 (NPT == 4 || (NPT == 8 && MODE == kFused)) && TNEED <= 512;
+                                 (NPT == 4 || NPT == 8) && TNEED <= 512;
     static constexpr int TCOLS = TNEED <= 32 ? 32 : (TNEED <= 64 ? 64 : (TNEED <= 128 ? 128 : (TNEED <= 256 ? 256 : 512)));
     // registers: the four N = 16 state-group warps of a CTA sit on the SM's four
     // sub-partitions, so 3 resident CTAs = 3 warps per sub-partition (<= 168
@@ -119,6 +119,7 @@ struct Cfg {
                                : ((T == 16 || KC == 16 || MODE == kLongFused) ? 3 : 2);
     static constexpr int MINB = (TMEM && 512 / TCOLS < MINB0) ? 512 / TCOLS : MINB0;
     static_assert(N % NPT == 0 && W <= 32, "state split");
+    static_assert(MODE != kLongFused || NPT % 4 == 0, "span checkpoints hold whole float4 groups");
 };
 
 // Shared-memory carve-up (bytes; every offset is a multiple of 16).
@@ -485,6 +486,7 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
                 for (int j = 0; j < NPT; ++j) gcar[j] = 0.f;
             }
             const int lo = (T > SPAN && ti == 0) ? SPAN : 0;   // the block's first span needs no checkpoint
+            // checkpoints [span][NPT/4][W][32] float4: a lane's NPT states in NPT/4 float4
             float4 *ck = reinterpret_cast<float4 *>(yrev) + warp * kCh + c;
             const int sb = (int)ti * (T / SPAN);   // span index of the tile's first token
 #pragma unroll
@@ -500,8 +502,12 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
                         gcar[2 * p] = g2.x;
                         gcar[2 * p + 1] = g2.y;
                     }
-                    if (t % SPAN == 0 && t < tlen && sb + t / SPAN >= 1)
-                        ck[(int64_t)(sb + t / SPAN - 1) * W * kCh] = make_float4(gcar[0], gcar[1], gcar[2], gcar[3]);
+                    if (t % SPAN == 0 && t < tlen && sb + t / SPAN >= 1) {
+#pragma unroll
+                        for (int q = 0; q < NPT / 4; ++q)
+                            ck[((int64_t)(sb + t / SPAN - 1) * (NPT / 4) + q) * W * kCh] =
+                                make_float4(gcar[4 * q], gcar[4 * q + 1], gcar[4 * q + 2], gcar[4 * q + 3]);
+                    }
                 }
             }
             continue;   // no output from this sweep
@@ -549,8 +555,12 @@ __global__ void __launch_bounds__(Cfg<N, MODE, KC, NPTV>::THREADS, Cfg<N, MODE, 
                 if (MODE == kLongFused) {   // the span's right-hand boundary condition
                     const int span = (int)ti * (T / SPAN) + sp;
                     if (span < nspan - 1) {
-                        const float4 g4 = reinterpret_cast<const float4 *>(yrev)[(int64_t)span * W * kCh + warp * kCh + c];
-                        gs[0] = g4.x; gs[1] = g4.y; gs[2] = g4.z; gs[3] = g4.w;
+#pragma unroll
+                        for (int q = 0; q < NPT / 4; ++q) {
+                            const float4 g4 = reinterpret_cast<const float4 *>(
+                                yrev)[((int64_t)span * (NPT / 4) + q) * W * kCh + warp * kCh + c];
+                            gs[4 * q] = g4.x; gs[4 * q + 1] = g4.y; gs[4 * q + 2] = g4.z; gs[4 * q + 3] = g4.w;
+                        }
                     }
                 }
                 if constexpr (CF::TMEM) {
