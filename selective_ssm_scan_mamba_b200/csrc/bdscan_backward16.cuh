@@ -219,6 +219,7 @@ __global__ void __launch_bounds__(128, 3) bdscan_bwd16_kernel(const BwdArgs a) {
         const IO *zs = reinterpret_cast<const IO *>(st) + 2 * TB * kCh + r0 * kCh;
         const IO *dys = reinterpret_cast<const IO *>(st) + 3 * TB * kCh + r0 * kCh;
         if (dvalid) {
+            const int64_t go0 = (b * L + t0 + warp * PER) * a.D + d;   // this warp's first token of the half
 #pragma unroll
             for (int i = 0; i < PER; ++i) {
                 const int t = warp * PER + i;
@@ -236,7 +237,7 @@ __global__ void __launch_bounds__(128, 3) bdscan_bwd16_kernel(const BwdArgs a) {
                 const float dxv = __fmaf_rn(q4.x, P, __fmul_rn(dfac, q4.z));
                 float ddl = __fmaf_rn(xv, P, Q);
                 if (a.dt_softplus) ddl = __fmul_rn(ddl, q4.w);
-                const int64_t go = (b * L + t0 + t) * a.D + d;
+                const int64_t go = go0 + i * a.D;
                 IO o;
                 from_f32(dxv, o);
                 static_cast<IO *>(a.dx)[go] = o;

@@ -105,6 +105,8 @@ STEP_CASES = [
     (1, 48, 64, 16, "bf16", True), (2, 32, 16, 64, "bf16", False), (1, 20, 24, 64, "f32", True),
     (1, 64, 32, 64, "bf16", True), (2, 100, 24, 16, "f32", False),
     (2, 16, 200, 64, "bf16", True), (3, 4, 72, 64, "f32", False),
+    # the block step of few rows at every compiled block length, partial channel tiles
+    (2, 4, 40, 16, "bf16", True), (1, 16, 24, 16, "bf16", False), (1, 32, 200, 16, "bf16", True),
 ]
 
 
