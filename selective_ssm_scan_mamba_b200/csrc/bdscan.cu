@@ -125,12 +125,14 @@ int launch_lag(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st) {
     return BDSCAN_OK;
 }
 
-// A block step (or a commit with y) of few rows at N = 16 (bdscan_step_kernel).
-template <class IO, int KC>
+// A block step (or a commit with y) of few rows at N = 16 (bdscan_step_kernel),
+// CW channels per CTA.
+template <class IO, int KC, int CW>
 int launch_step(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, bool pdl) {
     constexpr int T = KC > 0 ? KC : 32;
-    constexpr int smem = bdk::StepLayout<IO, T>::bytes;
-    auto kern = bdk::bdscan_step_kernel<IO, KC>;
+    constexpr int smem = bdk::StepLayout<IO, T, CW>::bytes;
+    constexpr int threads = bdk::StepCfg<CW>::THREADS;
+    auto kern = bdk::bdscan_step_kernel<IO, KC, CW>;
     static std::atomic<uint64_t> done_mask{0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
@@ -140,11 +142,11 @@ int launch_step(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, bool pdl
         if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
         done_mask.fetch_or(bit, std::memory_order_acq_rel);
     }
-    dim3 grid((unsigned)((a.D + bdk::kCh - 1) / bdk::kCh), (unsigned)batch, 1);
+    dim3 grid((unsigned)((a.D + CW - 1) / CW), (unsigned)batch, 1);
     if (pdl) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = grid;
-        cfg.blockDim = dim3(bdk::kStepThreads);
+        cfg.blockDim = dim3(threads);
         cfg.dynamicSmemBytes = smem;
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
@@ -155,23 +157,27 @@ int launch_step(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, bool pdl
         const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, a);
         if (le != cudaSuccess) { (void)cudaGetLastError(); g_last_cuda = le; return BDSCAN_ERR_CUDA; }
     } else {
-        kern<<<grid, bdk::kStepThreads, smem, st>>>(a);
+        kern<<<grid, threads, smem, st>>>(a);
     }
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
     return BDSCAN_OK;
 }
 
+int device_sm_count();
+
 template <class IO, int N>
 int dispatch_mode(int mode, const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1,
                   bool thin = false, bool pdl = false) {
     if constexpr (N == 16) {
         if (thin && mode == bdk::kFused) {   // one state per lane: the latency-bound small block step
+            // 16-channel CTAs when even those leave no SM with two of them
+            const bool half = batch * ((a.D + 15) / 16) <= device_sm_count();
             switch (a.K) {
-                case 4: return launch_step<IO, 4>(a, batch, st, pdl);
-                case 16: return launch_step<IO, 16>(a, batch, st, pdl);
-                case 32: return launch_step<IO, 32>(a, batch, st, pdl);
-                default: return launch_step<IO, 0>(a, batch, st, pdl);
+                case 4: return half ? launch_step<IO, 4, 16>(a, batch, st, pdl) : launch_step<IO, 4, 32>(a, batch, st, pdl);
+                case 16: return half ? launch_step<IO, 16, 16>(a, batch, st, pdl) : launch_step<IO, 16, 32>(a, batch, st, pdl);
+                case 32: return half ? launch_step<IO, 32, 16>(a, batch, st, pdl) : launch_step<IO, 32, 32>(a, batch, st, pdl);
+                default: return half ? launch_step<IO, 0, 16>(a, batch, st, pdl) : launch_step<IO, 0, 32>(a, batch, st, pdl);
             }
         }
     }

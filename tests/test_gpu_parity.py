@@ -107,6 +107,8 @@ STEP_CASES = [
     (2, 16, 200, 64, "bf16", True), (3, 4, 72, 64, "f32", False),
     # the block step of few rows at every compiled block length, partial channel tiles
     (2, 4, 40, 16, "bf16", True), (1, 16, 24, 16, "bf16", False), (1, 32, 200, 16, "bf16", True),
+    # rows of 16 channels more than the SMs, of 32 channels fewer: the 32-channel width
+    (1, 32, 2392, 16, "bf16", True), (1, 7, 2392, 16, "f32", False),
 ]
 
 
