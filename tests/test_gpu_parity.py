@@ -136,6 +136,30 @@ def test_block_step_and_commit_vs_oracle(bd, Bt, K, D, N, io, gated):
     assert torch.equal(cache2, cache)
 
 
+def test_block_step_channel_widths_agree_bitwise(bd):
+    """A block step of few rows runs 16 or 32 channels per CTA, chosen by the row
+    count. Channels are independent and both widths add a token's 16 per-state
+    partials in state order, so the same channels give the same bits whichever
+    width runs them: 2400 channels take the 32-channel width on 148 SMs (150
+    rows of 16), their first 1536 the 16-channel width (96 rows of 16)."""
+    K, wide, narrow = 32, 2400, 1536
+    s = make_case(977, 1, K, wide, 16, "bf16", gated=True, with_h0=True)
+    g = dev(s)
+    cut = lambda t: t[..., :narrow].contiguous()  # noqa: E731
+    cache_w, cache_n = g["h0"].clone(), g["h0"][:, :narrow].contiguous()
+    y_w = bd.block_step(g["x"], g["dt"], g["A"], g["B"], g["C"], g["Dskip"], cache_w, z=g["z"])
+    y_n = bd.block_step(cut(g["x"]), cut(g["dt"]), g["A"][:narrow].contiguous(), g["B"], g["C"],
+                        g["Dskip"][:narrow].contiguous(), cache_n, z=cut(g["z"]))
+    torch.cuda.synchronize()
+    assert torch.equal(y_w[..., :narrow], y_n)
+    yc_w = bd.commit_block(g["x"], g["dt"], g["A"], g["B"], g["C"], g["Dskip"], cache_w, z=g["z"], want_y=True)
+    yc_n = bd.commit_block(cut(g["x"]), cut(g["dt"]), g["A"][:narrow].contiguous(), g["B"], g["C"],
+                           g["Dskip"][:narrow].contiguous(), cache_n, z=cut(g["z"]), want_y=True)
+    torch.cuda.synchronize()
+    assert torch.equal(yc_w[..., :narrow], yc_n)
+    assert torch.equal(cache_w[:, :narrow], cache_n)
+
+
 @pytest.mark.parametrize("io,N,K", [("bf16", 16, 32), ("f32", 16, 16), ("bf16", 64, 16), ("f32", 64, 4)])
 def test_cache_exactness_on_gpu(bd, io, N, K):
     """Committing blocks one by one reproduces the one-shot prefill's boundary
