@@ -59,90 +59,27 @@ bool long_fused_fits(int64_t K) {
     return bdk::Layout<IO, N, bdk::kLongFused, 0>::base_bytes + long_fused_ck_bytes(K, N) <= (size_t)kMaxDynSmem;
 }
 
-// pdl: launch with programmatic stream serialisation, so that the kernel's
-// launch overlaps the end of the previous kernel in the stream (the kernel
-// waits for it before touching global memory).
-template <class IO, int N, int MODE, int KC, int NPTV = 4>
-int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1, bool pdl = false) {
-    using CF = bdk::Cfg<N, MODE, KC, NPTV>;
-    using LY = bdk::Layout<IO, N, MODE, KC, NPTV>;
-    const size_t smem = LY::base_bytes + (MODE == bdk::kLong ? (size_t)a.K * bdk::kCh * 4
-                                          : MODE == bdk::kLongFused ? long_fused_ck_bytes(a.K, N) : 0);
-    auto kern = bdk::bdscan_kernel<IO, N, MODE, KC, NPTV>;
-    // raise the dynamic shared-memory ceiling once per device
-    static std::atomic<uint64_t> done_mask{0};
+// Raise a kernel's dynamic shared-memory ceiling to cap bytes, once per device
+// (mask: the kernel's own record of the devices already done).
+template <class Kern>
+int smem_ceiling_once(Kern kern, int cap, std::atomic<uint64_t> &mask) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
     const uint64_t bit = 1ull << (dev & 63);
-    if (!(done_mask.load(std::memory_order_acquire) & bit)) {
-        const int cap = MODE == bdk::kLongFused ? kMaxDynSmem
-                                                 : LY::base_bytes + (MODE == bdk::kLong ? bdk::kLongSmemMax : 0);
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
+    if (!(mask.load(std::memory_order_acquire) & bit)) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
         if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
-        done_mask.fetch_or(bit, std::memory_order_acq_rel);
+        mask.fetch_or(bit, std::memory_order_acq_rel);
     }
-    dim3 grid((unsigned)((a.D + bdk::kCh - 1) / bdk::kCh), (unsigned)batch, gz);
-    if (pdl) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = grid;
-        cfg.blockDim = dim3(CF::THREADS);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, a);
-        if (le != cudaSuccess) { (void)cudaGetLastError(); g_last_cuda = le; return BDSCAN_ERR_CUDA; }
-    } else {
-        kern<<<grid, CF::THREADS, smem, st>>>(a);
-    }
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
     return BDSCAN_OK;
 }
 
-// The lagged whole-block pass (bdscan_lag_kernel).
-template <class IO, int N, int KC, int NPT>
-int launch_lag(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st) {
-    using CF = bdk::LagCfg<N, KC, NPT>;
-    using LY = bdk::LagLayout<IO, N, KC, NPT>;
-    auto kern = bdk::bdscan_lag_kernel<IO, N, KC, NPT>;
-    static std::atomic<uint64_t> done_mask{0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
-    const uint64_t bit = 1ull << (dev & 63);
-    if (!(done_mask.load(std::memory_order_acquire) & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::bytes);
-        if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
-        done_mask.fetch_or(bit, std::memory_order_acq_rel);
-    }
-    dim3 grid((unsigned)((a.D + bdk::kCh - 1) / bdk::kCh), (unsigned)batch, 1);
-    kern<<<grid, CF::THREADS, LY::bytes, st>>>(a);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
-    return BDSCAN_OK;
-}
-
-// A block step (or a commit with y) of few rows at N = 16 (bdscan_step_kernel),
-// CW channels per CTA.
-template <class IO, int KC, int CW>
-int launch_step(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, bool pdl) {
-    constexpr int T = KC > 0 ? KC : 32;
-    constexpr int smem = bdk::StepLayout<IO, T, CW>::bytes;
-    constexpr int threads = bdk::StepCfg<CW>::THREADS;
-    auto kern = bdk::bdscan_step_kernel<IO, KC, CW>;
-    static std::atomic<uint64_t> done_mask{0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
-    const uint64_t bit = 1ull << (dev & 63);
-    if (!(done_mask.load(std::memory_order_acquire) & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
-        done_mask.fetch_or(bit, std::memory_order_acq_rel);
-    }
-    dim3 grid((unsigned)((a.D + CW - 1) / CW), (unsigned)batch, 1);
+// Launch kern(a) on st. pdl: with programmatic stream serialisation, so that the
+// kernel's launch overlaps the end of the previous kernel in the stream (the
+// kernel waits for it before touching global memory).
+template <class Kern>
+int launch_kernel(Kern kern, dim3 grid, int threads, size_t smem, cudaStream_t st, bool pdl,
+                  const bdk::ScanArgs &a) {
     if (pdl) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = grid;
@@ -162,6 +99,49 @@ int launch_step(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, bool pdl
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
     return BDSCAN_OK;
+}
+
+// The fused, forward-only and long-block modes (bdscan_kernel).
+template <class IO, int N, int MODE, int KC, int NPTV = 4>
+int launch(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, unsigned gz = 1, bool pdl = false) {
+    using CF = bdk::Cfg<N, MODE, KC, NPTV>;
+    using LY = bdk::Layout<IO, N, MODE, KC, NPTV>;
+    const size_t smem = LY::base_bytes + (MODE == bdk::kLong ? (size_t)a.K * bdk::kCh * 4
+                                          : MODE == bdk::kLongFused ? long_fused_ck_bytes(a.K, N) : 0);
+    auto kern = bdk::bdscan_kernel<IO, N, MODE, KC, NPTV>;
+    static std::atomic<uint64_t> done_mask{0};
+    const int cap = MODE == bdk::kLongFused ? kMaxDynSmem : LY::base_bytes + (MODE == bdk::kLong ? bdk::kLongSmemMax : 0);
+    const int rc = smem_ceiling_once(kern, cap, done_mask);
+    if (rc != BDSCAN_OK) return rc;
+    const dim3 grid((unsigned)((a.D + bdk::kCh - 1) / bdk::kCh), (unsigned)batch, gz);
+    return launch_kernel(kern, grid, CF::THREADS, smem, st, pdl, a);
+}
+
+// The lagged whole-block pass (bdscan_lag_kernel).
+template <class IO, int N, int KC, int NPT>
+int launch_lag(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st) {
+    using CF = bdk::LagCfg<N, KC, NPT>;
+    using LY = bdk::LagLayout<IO, N, KC, NPT>;
+    auto kern = bdk::bdscan_lag_kernel<IO, N, KC, NPT>;
+    static std::atomic<uint64_t> done_mask{0};
+    const int rc = smem_ceiling_once(kern, LY::bytes, done_mask);
+    if (rc != BDSCAN_OK) return rc;
+    const dim3 grid((unsigned)((a.D + bdk::kCh - 1) / bdk::kCh), (unsigned)batch, 1);
+    return launch_kernel(kern, grid, CF::THREADS, LY::bytes, st, false, a);
+}
+
+// A block step (or a commit with y) of few rows at N = 16 (bdscan_step_kernel),
+// CW channels per CTA.
+template <class IO, int KC, int CW>
+int launch_step(const bdk::ScanArgs &a, int64_t batch, cudaStream_t st, bool pdl) {
+    constexpr int T = KC > 0 ? KC : 32;
+    constexpr int smem = bdk::StepLayout<IO, T, CW>::bytes;
+    auto kern = bdk::bdscan_step_kernel<IO, KC, CW>;
+    static std::atomic<uint64_t> done_mask{0};
+    const int rc = smem_ceiling_once(kern, smem, done_mask);
+    if (rc != BDSCAN_OK) return rc;
+    const dim3 grid((unsigned)((a.D + CW - 1) / CW), (unsigned)batch, 1);
+    return launch_kernel(kern, grid, bdk::StepCfg<CW>::THREADS, smem, st, pdl, a);
 }
 
 int device_sm_count();
@@ -429,15 +409,9 @@ int launch_bwd(const bdk::BwdArgs &a, int64_t batch, int64_t ct, void *dB, void 
     const bool b16 = N == 16 && a.K == 16;
     auto kern = b16 ? bdk::bdscan_bwd16_kernel<IO> : bdk::bdscan_bwd_kernel<IO, N>;
     const int smem = b16 ? bdk::Bwd16Layout<IO>::bytes : LY::bytes;
-    static std::atomic<uint64_t> done_mask{0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
-    const uint64_t bit = 1ull << ((2 * dev + (b16 ? 1 : 0)) & 63);
-    if (!(done_mask.load(std::memory_order_acquire) & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) { g_last_cuda = e; return BDSCAN_ERR_CUDA; }
-        done_mask.fetch_or(bit, std::memory_order_acq_rel);
-    }
+    static std::atomic<uint64_t> mask16{0}, mask_tiles{0};   // per kernel
+    const int rc = smem_ceiling_once(kern, smem, b16 ? mask16 : mask_tiles);
+    if (rc != BDSCAN_OK) return rc;
     if (batch > 0 && ct > 0) {
         kern<<<dim3((unsigned)ct, (unsigned)batch), CF::THREADS, smem, st>>>(a);
         cudaError_t e = cudaGetLastError();
