@@ -54,6 +54,9 @@ TRAIN_CASES = [
     # an odd number of 16-token blocks: the lagged schedule's last tile is half a tile
     (1, 112, 40, 64, 16, "bf16", True, True, True),
     (2, 80, 48, 16, 16, "f32", False, True, True),
+    # long blocks at N = 64 (8 states per lane): three spans, and a ragged last span
+    (2, 96, 24, 64, 48, "f32", False, False, True),
+    (1, 200, 40, 64, 100, "bf16", True, True, True),
     # long blocks whose span checkpoints do not fit in shared memory: the two-sweep path
     (1, 512, 16, 64, 512, "bf16", True, True, True),
     (1, 288, 16, 64, 288, "f32", False, True, True),
